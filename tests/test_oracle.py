@@ -1,0 +1,381 @@
+"""Pins for the CPU oracle, against things other than itself.
+
+* Two independent dense formulations (a numpy softmax written here, and
+  torch's scaled_dot_product_attention in fp64, a library routine).
+* Closed forms and special cases of softmax attention.
+* Invariants: causality, shift invariance, GQA equivalence, rotation invariance.
+* The e4m3 encoder/decoder against torch's float8_e4m3fn conversion (every
+  bf16 bit pattern in range) and the doubling rule the Lean P section states.
+* The fp32 Walsh-Hadamard butterfly against scipy's Sylvester matrix.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def dense_numpy(q, k, v, causal=True, scale=None):
+    """Independent dense formulation: materialise S, mask, softmax, multiply."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    kk = np.repeat(k, G, axis=2)
+    vv = np.repeat(v, G, axis=2)
+    s = np.einsum("bihc,bjhc->bhij", q, kk) * scale
+    if causal:
+        mask = np.triu(np.ones((N, N), dtype=bool), 1)
+        s = np.where(mask, -np.inf, s)
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=-1, keepdims=True)
+    return np.einsum("bhij,bjhc->bihc", p, vv)
+
+
+def sdpa_torch(q, k, v, causal=True, scale=None):
+    G = q.shape[2] // k.shape[2]
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(k).repeat_interleave(G, dim=2).permute(0, 2, 1, 3)
+    tv = torch.from_numpy(v).repeat_interleave(G, dim=2).permute(0, 2, 1, 3)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+SHAPES = [
+    # B, Hq, Hkv, N, d_qk, d_v
+    (1, 1, 1, 1, 128, 128),
+    (1, 1, 1, 37, 128, 128),
+    (2, 4, 2, 65, 16, 16),
+    (1, 8, 2, 130, 128, 128),
+    (1, 4, 1, 97, 192, 128),
+    (2, 2, 2, 256, 192, 128),
+    (1, 6, 3, 50, 8, 24),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("causal", [True, False])
+def test_matches_dense_numpy_and_torch_sdpa(shape, causal):
+    B, Hq, Hkv, N, dq, dv = shape
+    q = rand((B, N, Hq, dq), 1)
+    k = rand((B, N, Hkv, dq), 2)
+    v = rand((B, N, Hkv, dv), 3)
+    out, lse = oracle.attention(q, k, v, causal=causal)
+    ref = dense_numpy(q, k, v, causal=causal)
+    assert oracle.rel_rms(out, ref) < 1e-12
+    ref2 = sdpa_torch(q, k, v, causal=causal)
+    assert oracle.rel_rms(out, ref2) < 1e-12
+    # log-sum-exp of the scaled scores, computed densely
+    G = Hq // Hkv
+    s = np.einsum("bihc,bjhc->bihj", q, np.repeat(k, G, axis=2)) / np.sqrt(dq)
+    if causal:
+        s = np.where(np.triu(np.ones((N, N), dtype=bool), 1)[None, :, None, :], -np.inf, s)
+    mx = s.max(axis=-1)
+    ref_lse = mx + np.log(np.exp(s - mx[..., None]).sum(axis=-1))
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_row_subset_matches_full():
+    q, k, v = rand((2, 70, 4, 32), 4), rand((2, 70, 2, 32), 5), rand((2, 70, 2, 32), 6)
+    full, lse = oracle.attention(q, k, v)
+    rows = np.array([[0, 0, 0], [1, 3, 69], [0, 2, 33], [1, 1, 5]], dtype=np.int64)
+    sub, sub_lse = oracle.attention(q, k, v, rows=rows)
+    for r, (b, h, i) in enumerate(rows):
+        assert np.array_equal(sub[r], full[b, i, h])
+        assert sub_lse[r] == lse[b, i, h]
+
+
+def test_rejects_bad_rows():
+    q = rand((1, 4, 1, 8), 0)
+    with pytest.raises(ValueError):
+        oracle.attention(q, q, q, rows=np.array([[0, 0, 4]], dtype=np.int64))
+
+
+# ---------------------------------------------------------------- closed forms / special cases
+
+def test_single_token_returns_v0():
+    q, k, v = rand((1, 1, 2, 128), 7), rand((1, 1, 1, 128), 8), rand((1, 1, 1, 128), 9)
+    out, lse = oracle.attention(q, k, v)
+    assert np.array_equal(out[0, 0, 0], v[0, 0, 0]) and np.array_equal(out[0, 0, 1], v[0, 0, 0])
+    s = float(q[0, 0, 0] @ k[0, 0, 0]) / np.sqrt(128)
+    assert abs(lse[0, 0, 0] - s) < 1e-12
+
+
+def test_first_row_is_v0():
+    q, k, v = rand((1, 50, 2, 64), 10), rand((1, 50, 2, 64), 11), rand((1, 50, 2, 64), 12)
+    out, _ = oracle.attention(q, k, v)
+    np.testing.assert_array_equal(out[0, 0], v[0, 0])
+
+
+def test_equal_scores_give_prefix_mean():
+    N = 90
+    q = np.zeros((1, N, 1, 32))
+    k, v = rand((1, N, 1, 32), 13), rand((1, N, 1, 32), 14)
+    out, lse = oracle.attention(q, k, v)
+    prefix = np.cumsum(v[0, :, 0], axis=0) / np.arange(1, N + 1)[:, None]
+    np.testing.assert_allclose(out[0, :, 0], prefix, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse[0, :, 0], np.log(np.arange(1, N + 1)), rtol=1e-13)
+    # non-causal: every row is the global mean
+    out_nc, _ = oracle.attention(q, k, v, causal=False)
+    np.testing.assert_allclose(out_nc[0, :, 0], np.broadcast_to(v[0, :, 0].mean(0), (N, 32)),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_constant_v_gives_constant():
+    q, k = rand((1, 40, 2, 16), 15), rand((1, 40, 1, 16), 16)
+    v = np.full((1, 40, 1, 16), 3.25)
+    out, _ = oracle.attention(q, k, v)
+    np.testing.assert_allclose(out, 3.25, rtol=1e-14)
+
+
+def test_one_hot_v_recovers_probability_rows():
+    """V = identity over keys: O_i is row i of P; it sums to 1, is zero above the diagonal
+    and equals exp(s_ij - lse_i)."""
+    N = 48
+    q, k = rand((1, N, 1, 8), 17), rand((1, N, 1, 8), 18)
+    v = np.eye(N).reshape(1, N, 1, N)
+    P, lse = oracle.attention(q, k, v)
+    P = P[0, :, 0]
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=1e-13)
+    assert np.all(P[np.triu_indices(N, 1)] == 0.0)
+    s = (q[0, :, 0] @ k[0, :, 0].T) / np.sqrt(8)
+    expect = np.tril(np.exp(s - lse[0, :, 0][:, None]))
+    np.testing.assert_allclose(P, expect, rtol=1e-12, atol=1e-15)
+
+
+def test_two_key_closed_form():
+    """Row 1 with scores (0, ln 3): weights 1/4 and 3/4."""
+    d = 1
+    q = np.array([0.0, 1.0]).reshape(1, 2, 1, d)
+    k = np.array([0.0, np.log(3.0)]).reshape(1, 2, 1, d)
+    v = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 2, 1, 2)
+    out, lse = oracle.attention(q, k, v, softmax_scale=1.0)
+    np.testing.assert_allclose(out[0, 1, 0], [0.25, 0.75], rtol=1e-14)
+    np.testing.assert_allclose(lse[0, 1, 0], np.log(4.0), rtol=1e-14)
+
+
+def test_large_scale_selects_argmax():
+    N = 33
+    q, k, v = rand((1, N, 1, 16), 19), rand((1, N, 1, 16), 20), rand((1, N, 1, 16), 21)
+    out, _ = oracle.attention(q, k, v, softmax_scale=1e4)
+    s = q[0, :, 0] @ k[0, :, 0].T
+    for i in range(N):
+        j = int(np.argmax(s[i, : i + 1]))
+        np.testing.assert_allclose(out[0, i, 0], v[0, j, 0], rtol=1e-9, atol=1e-9)
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_causality_bitwise():
+    N = 64
+    q, k, v = rand((1, N, 2, 32), 22), rand((1, N, 1, 32), 23), rand((1, N, 1, 32), 24)
+    base, _ = oracle.attention(q, k, v)
+    for i in (0, 10, 40, 62):
+        k2, v2 = k.copy(), v.copy()
+        k2[:, i + 1:] = rand(k2[:, i + 1:].shape, 100 + i)
+        v2[:, i + 1:] = rand(v2[:, i + 1:].shape, 200 + i)
+        out, _ = oracle.attention(q, k2, v2)
+        assert np.array_equal(out[:, : i + 1], base[:, : i + 1])
+
+
+def test_row_shift_invariance():
+    """Adding c_i to every score of row i (an extra dim: q gets c_i, k gets 1) leaves O unchanged."""
+    N, d = 40, 16
+    q, k, v = rand((1, N, 1, d), 25), rand((1, N, 1, d), 26), rand((1, N, 1, d), 27)
+    c = 5.0 * rand((1, N, 1, 1), 28)
+    qa = np.concatenate([q, c], axis=-1)
+    ka = np.concatenate([k, np.ones((1, N, 1, 1))], axis=-1)
+    a, _ = oracle.attention(q, k, v, softmax_scale=0.3)
+    b, _ = oracle.attention(qa, ka, v, softmax_scale=0.3)
+    np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-12)
+
+
+def test_gqa_equals_explicit_replication():
+    q, k, v = rand((2, 30, 8, 16), 29), rand((2, 30, 2, 16), 30), rand((2, 30, 2, 16), 31)
+    a, la = oracle.attention(q, k, v)
+    b, lb = oracle.attention(q, np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2))
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_orthogonal_rotation_invariance():
+    """Rotating Q and K by the same orthonormal Hadamard matrix leaves attention unchanged."""
+    H = scipy.linalg.hadamard(128) / np.sqrt(128.0)
+    q, k, v = rand((1, 60, 2, 128), 32), rand((1, 60, 1, 128), 33), rand((1, 60, 1, 128), 34)
+    a, _ = oracle.attention(q, k, v)
+    b, _ = oracle.attention(q @ H.T, k @ H.T, v)
+    assert oracle.rel_rms(b, a) < 1e-12
+
+
+# ---------------------------------------------------------------- e4m3 format
+
+def all_bf16_values():
+    bits = np.arange(1 << 16, dtype=np.uint32) << 16
+    vals = bits.view(np.float32)
+    return vals[np.isfinite(vals)]
+
+
+def test_e4m3_encode_matches_torch_on_every_bf16_in_range():
+    x = all_bf16_values()
+    x = x[np.abs(x) <= 448.0]
+    ours = oracle.e4m3_encode(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_encode_matches_torch_on_random_fp32():
+    rng = np.random.default_rng(35)
+    bits = rng.integers(0, 1 << 32, size=2_000_000, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    x = x[np.isfinite(x) & (np.abs(x) <= 448.0)]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(x), ref)
+
+
+def test_e4m3_saturates_and_nan():
+    x = np.array([448.0, 463.99, 464.0, 470.0, 1e30, -1e30, np.nan, -0.0, 0.0], dtype=np.float32)
+    c = oracle.e4m3_encode(x)
+    assert list(c[:6]) == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+    assert c[6] & 0x7F == 0x7F
+    assert c[7] == 0x80 and c[8] == 0x00
+
+
+def test_e4m3_decode_matches_torch_for_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    both_nan = np.isnan(ours) & np.isnan(ref)
+    assert np.array_equal(ours[~both_nan], ref[~both_nan]) and both_nan.sum() == 2
+
+
+def test_e4m3_code_grows_by_fixed_step_per_doubling():
+    facts = json.load(open(os.path.join(HERE, "golden", "e4m3_lean_p_facts.json")))
+    step = facts["doubling_code_step"]
+    # every normal value whose double is still finite
+    codes = np.arange(8, 0x7F - step, dtype=np.uint8)
+    vals = oracle.e4m3_decode(codes).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_encode(2 * vals).astype(int) - codes.astype(int),
+                          np.full(codes.shape, step))
+    # code(2^x) is 8x + a constant for integer x across the normal range
+    xs = np.arange(-6, 9)
+    c = oracle.e4m3_encode(np.ldexp(np.float32(1.0), xs)).astype(int)
+    assert np.all(c - step * xs == c[0] - step * xs[0])
+
+
+def test_decode_encode_roundtrip():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    back = oracle.e4m3_encode(oracle.e4m3_decode(codes).astype(np.float32))
+    # +0 and -0 both round trip bit-exactly
+    assert np.array_equal(back, codes)
+
+
+# ---------------------------------------------------------------- Hadamard
+
+@pytest.mark.parametrize("n", [2, 8, 64, 128])
+def test_fwht_matches_sylvester_matrix(n):
+    x = rand((50, n), 36).astype(np.float32)
+    ref = x.astype(np.float64) @ scipy.linalg.hadamard(n).T
+    got = oracle.fwht(x).astype(np.float64)
+    assert np.max(np.abs(got - ref)) <= 1e-5 * np.max(np.abs(ref))
+
+
+def test_hadamard_rotation_is_orthonormal():
+    x = rand((20, 3, 128), 37).astype(np.float32)
+    y = oracle.hadamard_rotate(x)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-5)
+    np.testing.assert_allclose(oracle.hadamard_rotate(y), x, rtol=1e-4, atol=1e-5)
+    x192 = rand((5, 192), 38).astype(np.float32)
+    H = scipy.linalg.block_diag(scipy.linalg.hadamard(128) / np.sqrt(128), scipy.linalg.hadamard(64) / 8)
+    np.testing.assert_allclose(oracle.hadamard_rotate(x192), x192.astype(np.float64) @ H.T,
+                               rtol=1e-5, atol=1e-5)
+
+
+def test_fwht_butterfly_is_fp32_exact_sequence():
+    """Each stage is one IEEE fp32 add or subtract: redoing stage by stage in float64 and
+    rounding to fp32 after every stage gives the same bits."""
+    x = rand((8, 128), 39).astype(np.float32)
+    y = x.astype(np.float64)
+    h = 1
+    while h < 128:
+        y = y.reshape(8, 128 // (2 * h), 2, h)
+        y = np.stack([y[:, :, 0] + y[:, :, 1], y[:, :, 0] - y[:, :, 1]], axis=2)
+        y = y.astype(np.float32).astype(np.float64).reshape(8, 128)
+        h *= 2
+    assert np.array_equal(y.astype(np.float32), oracle.fwht(x))
+
+
+# ---------------------------------------------------------------- quantizer
+
+def test_quantize_per_head_maps_amax_to_448_and_bounds_error():
+    x = (rand((2, 300, 3, 128), 40) * np.array([0.1, 1.0, 30.0])[None, None, :, None]).astype(np.float32)
+    codes, scales = oracle.quantize_fp8(x, "head")
+    assert scales.shape == (2, 3) and codes.dtype == np.uint8
+    amax = np.abs(x).max(axis=(1, 3))
+    np.testing.assert_array_equal(scales, (amax / np.float32(448)).astype(np.float32))
+    dq = oracle.dequantize(codes, scales, "head")
+    # e4m3 RNE: relative error <= 2^-4 in the normal range, absolute <= 2^-10 * scale below it
+    err = np.abs(dq - x)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, scales[:, None, :, None] * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(err <= bound)
+    # the largest magnitude of each head is exactly +-448 (code 0x7E / 0xFE)
+    for b in range(2):
+        for h in range(3):
+            flat = np.abs(x[b, :, h]).ravel()
+            c = codes[b, :, h].ravel()[np.argmax(flat)]
+            assert c & 0x7F == 0x7E
+
+
+def test_quantize_per_block_scales():
+    x = rand((1, 300, 2, 128), 41).astype(np.float32)
+    x[:, 128:256] *= 50.0
+    codes, scales = oracle.quantize_fp8(x, "block")
+    assert scales.shape == (1, 2, 3)
+    for blk, sl in enumerate([slice(0, 128), slice(128, 256), slice(256, 300)]):
+        amax = np.abs(x[:, sl]).max(axis=(1, 3))
+        np.testing.assert_array_equal(scales[:, :, blk], amax / np.float32(448))
+    dq = oracle.dequantize(codes, scales, "block")
+    assert oracle.rel_rms(dq, x) < 0.04
+
+
+def test_quantize_zero_tensor():
+    codes, scales = oracle.quantize_fp8(np.zeros((1, 10, 2, 128), np.float32), "head")
+    assert np.all(codes == 0) and np.all(scales == 1.0)
+
+
+def test_quantize_with_hadamard_uses_rotated_values():
+    x = rand((1, 64, 1, 128), 42).astype(np.float32)
+    c1, s1 = oracle.quantize_fp8(x, "head", hadamard=True)
+    c2, s2 = oracle.quantize_fp8(oracle.hadamard_rotate(x), "head", hadamard=False)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def test_hadamard_reduces_fp8_error_with_outlier_channels():
+    """With a few large-gain channels, rotating Q and K before quantising lowers the attention
+    error against unquantised fp64 (the direction the accuracy section reports)."""
+    rng = np.random.default_rng(43)
+    N, d = 256, 128
+    gain = np.ones(d)
+    gain[rng.choice(d, 3, replace=False)] = 15.0
+    q = (rng.standard_normal((1, N, 1, d)) * gain).astype(np.float32)
+    k = (rng.standard_normal((1, N, 1, d)) * gain).astype(np.float32)
+    v = rng.standard_normal((1, N, 1, d)).astype(np.float32)
+    ref, _ = oracle.attention(q, k, v, softmax_scale=1.0 / np.sqrt(d) / 8)
+    errs = []
+    for had in (False, True):
+        cq, sq = oracle.quantize_fp8(q, "head", had)
+        ck, sk = oracle.quantize_fp8(k, "head", had)
+        cv, sv = oracle.quantize_fp8(v, "head", False)
+        out, _ = oracle.attention(oracle.dequantize(cq, sq), oracle.dequantize(ck, sk),
+                                  oracle.dequantize(cv, sv), softmax_scale=1.0 / np.sqrt(d) / 8)
+        errs.append(oracle.rel_rms(out, ref))
+    assert errs[1] < errs[0]
