@@ -1,0 +1,16 @@
+"""Causal prefill attention forward for NVIDIA B200 (sm_100a), BF16 and FP8 e4m3.
+
+The compute lives in libb200attn.so (hand-written CUDA for sm_100a behind the
+C ABI in include/b200attn.h); this package is its thin Python binding.
+"""
+from ._binding import (  # noqa: F401
+    B200AttnError,
+    LIB_PATH,
+    attn_func,
+    attn_fwd,
+    check,
+    load_library,
+    quantize_fp8,
+    quantize_workspace_bytes,
+    version,
+)

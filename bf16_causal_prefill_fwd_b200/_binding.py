@@ -1,0 +1,185 @@
+"""ctypes binding of libb200attn (include/b200attn.h). Argument marshalling only:
+every step of attention and quantisation runs in the library's CUDA kernels.
+
+PyTorch supplies device memory and the current stream; nothing here computes.
+If the library is not built, every call raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libb200attn.so")
+
+BF16 = 0
+FP8_E4M3 = 1
+SCALE_PER_HEAD = 0
+SCALE_PER_BLOCK = 1
+_GRAN = {"head": SCALE_PER_HEAD, "block": SCALE_PER_BLOCK}
+BLOCK = 128
+
+_lib = None
+
+
+class B200AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        msg = _lib.b200attn_strerror(code).decode() if _lib is not None else "library not loaded"
+        super().__init__(f"{what}: {msg} (status {code})")
+        self.code = code
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libb200attn.so (raises if it is missing: build it with
+    ``python -m bf16_causal_prefill_fwd_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing; build it with `python -m bf16_causal_prefill_fwd_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.b200attn_fwd.restype = i
+    lib.b200attn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, vp, vp, i, f, vp, vp]
+    lib.b200attn_quantize_workspace_bytes.restype = sz
+    lib.b200attn_quantize_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.b200attn_quantize_fp8.restype = i
+    lib.b200attn_quantize_fp8.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
+    lib.b200attn_check.restype = i
+    lib.b200attn_check.argtypes = [vp]
+    lib.b200attn_strerror.restype = ctypes.c_char_p
+    lib.b200attn_strerror.argtypes = [i]
+    lib.b200attn_version.restype = i
+    lib.b200attn_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_cuda_contig(name, t):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous ([B, N, H, d], d fastest)")
+
+
+def _is_fp8(t):
+    return t.dtype in (torch.float8_e4m3fn, torch.uint8)
+
+
+def attn_fwd(q, k, v, *, causal: bool = True, softmax_scale: float | None = None,
+             q_scale=None, k_scale=None, v_scale=None, scale_granularity: str = "head",
+             out=None, return_lse: bool = False, stream=None):
+    """O = softmax(s Q K^T [+ causal mask]) V via b200attn_fwd.
+
+    q [B,N,Hq,d_qk], k [B,N,Hkv,d_qk], v [B,N,Hkv,d_v]: bf16, or e4m3 codes
+    (torch.float8_e4m3fn or uint8) with fp32 scales. Returns bf16 [B,N,Hq,d_v]
+    (and fp32 lse [B,Hq,N] if ``return_lse``).
+    """
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_cuda_contig(name, t)
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be 4-D [B, N, H, d]")
+    fp8 = _is_fp8(q)
+    if fp8 != _is_fp8(k) or fp8 != _is_fp8(v) or (not fp8 and not (q.dtype == k.dtype == v.dtype == torch.bfloat16)):
+        raise ValueError("q, k, v must all be bf16 or all e4m3")
+    B, N, Hq, d_qk = q.shape
+    Hkv, d_v = k.shape[2], v.shape[3]
+    if k.shape != (B, N, Hkv, d_qk) or v.shape != (B, N, Hkv, d_v):
+        raise ValueError("shape mismatch between q, k and v")
+    if out is None:
+        out = torch.empty((B, N, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    else:
+        _check_cuda_contig("out", out)
+        if out.dtype != torch.bfloat16 or out.shape != (B, N, Hq, d_v):
+            raise ValueError("out must be bf16 [B, N, Hq, d_v]")
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if return_lse else None
+    if fp8:
+        for name, s in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+            if s is None:
+                raise ValueError(f"{name} is required for e4m3 inputs")
+            _check_cuda_contig(name, s)
+            if s.dtype != torch.float32:
+                raise ValueError(f"{name} must be fp32")
+    rc = lib.b200attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d_qk, d_v, 1 if causal else 0,
+        FP8_E4M3 if fp8 else BF16,
+        _ptr(q_scale) if fp8 else None, _ptr(k_scale) if fp8 else None, _ptr(v_scale) if fp8 else None,
+        _GRAN[scale_granularity], float(softmax_scale) if softmax_scale else 0.0,
+        _ptr(lse), _stream_handle(stream))
+    if rc != 0:
+        raise B200AttnError(rc, "b200attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def quantize_workspace_bytes(B, N, H, d, granularity="head") -> int:
+    return int(load_library().b200attn_quantize_workspace_bytes(B, N, H, d, _GRAN[granularity]))
+
+
+def quantize_fp8(x, *, granularity: str = "head", hadamard: bool = False, out=None, scale=None,
+                 workspace=None, stream=None):
+    """bf16 [B,N,H,d] -> (e4m3 codes as torch.float8_e4m3fn [B,N,H,d], fp32 scales).
+
+    Scales are [B,H] (granularity "head") or [B,H,ceil(N/128)] ("block"); a
+    code c stands for decode(c) * scale.
+    """
+    lib = load_library()
+    _check_cuda_contig("x", x)
+    if x.dtype != torch.bfloat16 or x.dim() != 4:
+        raise ValueError("x must be bf16 [B, N, H, d]")
+    B, N, H, d = x.shape
+    if out is None:
+        out = torch.empty((B, N, H, d), dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        shape = (B, H) if granularity == "head" else (B, H, math.ceil(N / BLOCK))
+        scale = torch.empty(shape, dtype=torch.float32, device=x.device)
+    need = quantize_workspace_bytes(B, N, H, d, granularity)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.b200attn_quantize_fp8(_ptr(x), _ptr(out), _ptr(scale), B, N, H, d, _GRAN[granularity],
+                                   1 if hadamard else 0, _ptr(workspace), wbytes, _stream_handle(stream))
+    if rc != 0:
+        raise B200AttnError(rc, "b200attn_quantize_fp8")
+    return out, scale
+
+
+def attn_func(q, k, v, softmax_scale: float | None = None, causal: bool = True, *, fp8: bool = False,
+              hadamard: bool = False, granularity: str = "head", return_lse: bool = False, stream=None):
+    """flash_attn_func-style call on bf16 [B,N,H,d] tensors.
+
+    With ``fp8=True`` Q, K and V are first quantised to e4m3 (Q and K
+    optionally Hadamard-rotated, which leaves Q K^T unchanged), then the FP8
+    kernel runs.
+    """
+    if not fp8:
+        return attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale, return_lse=return_lse,
+                        stream=stream)
+    q8, sq = quantize_fp8(q, granularity=granularity, hadamard=hadamard, stream=stream)
+    k8, sk = quantize_fp8(k, granularity=granularity, hadamard=hadamard, stream=stream)
+    v8, sv = quantize_fp8(v, granularity=granularity, hadamard=False, stream=stream)
+    return attn_fwd(q8, k8, v8, causal=causal, softmax_scale=softmax_scale, q_scale=sq, k_scale=sk,
+                    v_scale=sv, scale_granularity=granularity, return_lse=return_lse, stream=stream)
+
+
+def check(stream=None) -> int:
+    """Synchronise the stream and return/clear the library's device status word (0 = ok)."""
+    return int(load_library().b200attn_check(_stream_handle(stream)))
+
+
+def version() -> int:
+    return int(load_library().b200attn_version())

@@ -1,0 +1,215 @@
+// C-ABI entry points of libb200attn (declared in include/b200attn.h):
+// argument validation, TMA tensor-map encoding, kernel selection and launch.
+// Everything the operation computes runs in the kernels of attn_fwd_kernel.cuh
+// and quant_kernel.cuh; this file only marshals.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/b200attn.h"
+#include "attn_fwd_kernel.cuh"
+#include "quant_kernel.cuh"
+
+namespace {
+
+using b200::AttnCfg;
+using b200::AttnParams;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B, N, H, d] row-major tensor as a 4-D TMA map {d, H, N, B}; box = {inner, 1, 128, 1},
+// 128-byte swizzle. Out-of-range rows and columns read as zero.
+bool make_tmap(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, int N, int B) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t esz = fp8 ? 1 : 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * esz, (cuuint64_t)H * d * esz, (cuuint64_t)N * H * d * esz};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / esz), 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                         const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_ok(int* sm_count) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return B200ATTN_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return B200ATTN_ERR_CUDA;
+  if (major != 10 || minor != 0) return B200ATTN_ERR_UNSUPPORTED;
+  return B200ATTN_OK;
+}
+
+template <int DQK, int DV, bool FP8>
+int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
+                cudaStream_t stream) {
+  using C = AttnCfg<DQK, DV, FP8>;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, FP8, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, FP8, d_qk, p.Hkv, p.N, p.B) ||
+      !make_tmap(&tv, v, FP8, d_v, p.Hkv, p.N, p.B))
+    return B200ATTN_ERR_CUDA;
+  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return B200ATTN_ERR_CUDA;
+  const int grid = p.n_units < sm_count ? p.n_units : sm_count;
+  kern<<<grid, b200::kAttnThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+template <int D, bool HAD>
+int launch_quant(const void* x, void* y, float* scale, int B, int N, int H, int gran, void* ws, cudaStream_t stream) {
+  const int nblk = (N + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  const dim3 grid(nblk, H, B);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* yb = static_cast<uint8_t*>(y);
+  if (gran == B200ATTN_SCALE_PER_HEAD) {
+    float* partial = static_cast<float*>(ws);
+    b200::quant_absmax_kernel<D, HAD><<<grid, b200::kQuantThreads, 0, stream>>>(xb, partial, N, H);
+    b200::quant_encode_kernel<D, HAD, true><<<grid, b200::kQuantThreads, 0, stream>>>(xb, yb, scale, partial, N, H);
+  } else {
+    b200::quant_encode_kernel<D, HAD, false><<<grid, b200::kQuantThreads, 0, stream>>>(xb, yb, scale, nullptr, N, H);
+  }
+  return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N, int d_qk,
+                 int d_v, int causal, int dtype, const float* q_scale, const float* k_scale, const float* v_scale,
+                 int scale_granularity, float softmax_scale, float* lse, void* stream) {
+  if (!q || !k || !v || !o) return B200ATTN_ERR_INVALID;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d_qk < 1 || d_v < 1) return B200ATTN_ERR_INVALID;
+  if (Hq % Hkv != 0) return B200ATTN_ERR_INVALID;
+  if (causal != 0 && causal != 1) return B200ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return B200ATTN_ERR_INVALID;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return B200ATTN_ERR_INVALID;
+  if (dtype != B200ATTN_BF16 && dtype != B200ATTN_FP8_E4M3) return B200ATTN_ERR_UNSUPPORTED;
+  if (!(d_v == 128 && (d_qk == 128 || d_qk == 192))) return B200ATTN_ERR_UNSUPPORTED;
+  if (!(std::isfinite(softmax_scale))) return B200ATTN_ERR_INVALID;
+  const bool fp8 = dtype == B200ATTN_FP8_E4M3;
+  if (fp8) {
+    if (!q_scale || !k_scale || !v_scale) return B200ATTN_ERR_INVALID;
+    if (scale_granularity != B200ATTN_SCALE_PER_HEAD) return B200ATTN_ERR_UNSUPPORTED;
+  }
+  // index arithmetic inside the kernels is 32-bit over (b, n, h) rows
+  if (static_cast<int64_t>(B) * N * (Hq > Hkv ? Hq : Hkv) >= (int64_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
+  int sm_count = 0;
+  const int dev_rc = device_ok(&sm_count);
+  if (dev_rc != B200ATTN_OK) return dev_rc;
+
+  AttnParams p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.G = Hq / Hkv;
+  p.n_kv = (N + b200::kBN - 1) / b200::kBN;
+  p.n_pairs = (p.n_kv + 1) / 2;
+  const int64_t units = static_cast<int64_t>(B) * Hq * p.n_pairs;
+  if (units >= (int64_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
+  p.n_units = static_cast<int>(units);
+  p.causal = causal;
+  p.per_block = scale_granularity == B200ATTN_SCALE_PER_BLOCK;
+  const double s = softmax_scale > 0.0f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d_qk));
+  p.scale_log2 = static_cast<float>(s * 1.4426950408889634);
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if (!fp8) {
+    if (d_qk == 128) return launch_attn<128, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
+    return launch_attn<192, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
+  }
+  if (d_qk == 128) return launch_attn<128, 128, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+  return launch_attn<192, 128, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+}
+
+size_t b200attn_quantize_workspace_bytes(int B, int N, int H, int d, int granularity) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return 0;
+  if (granularity != B200ATTN_SCALE_PER_HEAD) return 0;
+  const size_t nblk = (static_cast<size_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  return static_cast<size_t>(B) * H * nblk * sizeof(float);
+}
+
+int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale, int B, int N, int H, int d, int granularity,
+                          int hadamard, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !x_fp8 || !scale) return B200ATTN_ERR_INVALID;
+  if (B < 1 || N < 1 || H < 1 || d < 1) return B200ATTN_ERR_INVALID;
+  if (granularity != B200ATTN_SCALE_PER_HEAD && granularity != B200ATTN_SCALE_PER_BLOCK)
+    return B200ATTN_ERR_UNSUPPORTED;
+  if (hadamard != 0 && hadamard != 1) return B200ATTN_ERR_INVALID;
+  if (d != 128 && d != 192) return B200ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(x_fp8) || (reinterpret_cast<uintptr_t>(scale) & 3u)) return B200ATTN_ERR_INVALID;
+  const int64_t nblk = (static_cast<int64_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  if (nblk > 0x7fffffff || H > 65535 || B > 65535) return B200ATTN_ERR_UNSUPPORTED;
+  const size_t need = b200attn_quantize_workspace_bytes(B, N, H, d, granularity);
+  if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 3u)))
+    return B200ATTN_ERR_WORKSPACE;
+  int sm_count = 0;
+  const int dev_rc = device_ok(&sm_count);
+  if (dev_rc != B200ATTN_OK) return dev_rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return hadamard ? launch_quant<128, true>(x, x_fp8, scale, B, N, H, granularity, workspace, st)
+                    : launch_quant<128, false>(x, x_fp8, scale, B, N, H, granularity, workspace, st);
+  return hadamard ? launch_quant<192, true>(x, x_fp8, scale, B, N, H, granularity, workspace, st)
+                  : launch_quant<192, false>(x, x_fp8, scale, B, N, H, granularity, workspace, st);
+}
+
+int b200attn_check(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return B200ATTN_ERR_CUDA;
+  int status = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&status, b200::g_b200attn_status, sizeof(int)) != cudaSuccess) return B200ATTN_ERR_CUDA;
+  if (status != 0 && cudaMemcpyToSymbol(b200::g_b200attn_status, &zero, sizeof(int)) != cudaSuccess)
+    return B200ATTN_ERR_CUDA;
+  return status;
+}
+
+const char* b200attn_strerror(int code) {
+  switch (code) {
+    case B200ATTN_OK: return "ok";
+    case B200ATTN_ERR_INVALID: return "invalid argument";
+    case B200ATTN_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case B200ATTN_ERR_CUDA: return "CUDA runtime or driver error";
+    case B200ATTN_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case B200ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int b200attn_version(void) { return B200ATTN_VERSION; }
+
+}  // extern "C"

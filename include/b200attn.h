@@ -1,0 +1,167 @@
+/*
+ * b200attn -- causal prefill attention forward for NVIDIA B200 (sm_100a),
+ * BF16 and FP8 e4m3, head dim 128 (with grouped-query attention) and the MLA
+ * shape (qk dim 192, v dim 128).
+ *
+ * The operation. For every batch b, query head h_q and query position i:
+ *
+ *     O[b,i,h_q,:] = softmax_j( s * Q[b,i,h_q,:] . K[b,j,h_k,:] ) V[b,j,h_k,:]
+ *     with j <= i (causal) or j < N (non-causal), h_k = h_q / (Hq / Hkv).
+ *
+ * The pages this library follows define it as causal forward ("prefill")
+ * attention in FP8 e4m3 and BF16 at head dim 128 and at the 192/128 MLA head
+ * shape, as a drop-in for flash_attn_func: "Zyphra 开源 ZYFA：面向 AMD MI355X 的
+ * FP8 FlashAttention，最高提速 1.76 倍", TL;DR; "Zyphra Says Its AMD MI355X
+ * Attention Kernel Is 1.76x Faster", "What Zyphra Reported". The FP8 path keeps
+ * FP32 accumulation and per-head scale factors: "Zyphra ZYFA: 1.76x FP8
+ * FlashAttention Speedup on AMD MI355X", "ZYFA's performance and accuracy
+ * data".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors use the flash_attn_func layout, row-major [B, N, H, d] with d
+ *   fastest and no padding. Pointers are DEVICE pointers on the current CUDA
+ *   device, 16-byte aligned, owned by the caller, and must not alias.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream). All work is
+ *   enqueued on it; no entry point synchronises, except b200attn_check.
+ * - Return value: 0 on success, or a negative b200attn_status. On an argument
+ *   error nothing is launched and no output is touched.
+ * - A kernel never traps. Every wait inside a kernel is bounded (about two
+ *   seconds); if one runs out, the kernel stops, frees its tensor memory,
+ *   records B200ATTN_ERR_TIMEOUT in a device status word and returns. The
+ *   status word is read (and cleared) by b200attn_check.
+ * - The library holds no device memory of its own beyond that status word.
+ */
+#ifndef B200ATTN_H_
+#define B200ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define B200ATTN_VERSION 100 /* 1.0.0 */
+
+typedef enum {
+  B200ATTN_OK = 0,
+  B200ATTN_ERR_INVALID = -1,     /* bad argument: NULL pointer, bad size, misaligned pointer */
+  B200ATTN_ERR_UNSUPPORTED = -2, /* well-formed but not implemented (head dims, device) */
+  B200ATTN_ERR_CUDA = -3,        /* the CUDA runtime or driver reported an error */
+  B200ATTN_ERR_TIMEOUT = -4,     /* a kernel's bounded wait ran out (device status word) */
+  B200ATTN_ERR_WORKSPACE = -5    /* workspace missing or smaller than required */
+} b200attn_status;
+
+/* dtype of Q, K and V. */
+enum { B200ATTN_BF16 = 0, B200ATTN_FP8_E4M3 = 1 };
+
+/* Granularity of FP8 scale factors. */
+enum {
+  B200ATTN_SCALE_PER_HEAD = 0, /* one fp32 scale per (b, h): array [B, H] */
+  B200ATTN_SCALE_PER_BLOCK = 1 /* one fp32 scale per (b, h, 128-token block): [B, H, ceil(N/128)] */
+};
+
+/*
+ * b200attn_fwd -- causal (or full) softmax attention forward.
+ *
+ * Defined by: "Zyphra 开源 ZYFA …", TL;DR (causal forward prefill, e4m3 and
+ * BF16, head dim 128 and 192/128, flash_attn_func drop-in) and "ZYFA 如何工作？"
+ * (FP8 probabilities, divide by the row sum of the probabilities actually used).
+ *
+ * q      [B, N, Hq,  d_qk]  bf16, or e4m3 codes when dtype == FP8_E4M3
+ * k      [B, N, Hkv, d_qk]  same dtype as q
+ * v      [B, N, Hkv, d_v]   same dtype as q
+ * o      [B, N, Hq,  d_v]   bf16 output (always bf16)
+ * B, N   batch and sequence length (Nq = Nk = N), B >= 1, N >= 1
+ * Hq,Hkv query and key/value heads; Hq % Hkv == 0; query head h uses key/value
+ *        head h / (Hq/Hkv)
+ * d_qk, d_v  supported pairs: (128, 128) and (192, 128)
+ * causal 1: key j is visible to query i iff j <= i; 0: every key is visible
+ * dtype  B200ATTN_BF16 or B200ATTN_FP8_E4M3
+ * q_scale, k_scale, v_scale
+ *        FP8 only (ignored for BF16, may be NULL): device fp32 dequantisation
+ *        scales; a code c of tensor X stands for decode(c) * X_scale. Shape
+ *        [B, H] for SCALE_PER_HEAD; [B, H, ceil(N/128)] for SCALE_PER_BLOCK
+ *        (H = Hq for q, Hkv for k and v).
+ * scale_granularity  B200ATTN_SCALE_PER_HEAD or B200ATTN_SCALE_PER_BLOCK
+ * softmax_scale  s; a value <= 0 selects 1/sqrt(d_qk)
+ * lse    optional (NULL allowed) fp32 [B, Hq, N]: natural-log sum over visible
+ *        keys of exp(s * q.k) for each query row
+ * stream cudaStream_t
+ *
+ * Errors: INVALID for NULL q/k/v/o, non-positive sizes, Hq % Hkv != 0,
+ * misaligned pointers, or missing FP8 scales; UNSUPPORTED for other head dims,
+ * a device that is not compute capability 10.0, or an unknown dtype or
+ * granularity; CUDA when the launch fails.
+ */
+int b200attn_fwd(const void* q, const void* k, const void* v, void* o,
+                 int B, int Hq, int Hkv, int N, int d_qk, int d_v,
+                 int causal, int dtype,
+                 const float* q_scale, const float* k_scale, const float* v_scale,
+                 int scale_granularity, float softmax_scale,
+                 float* lse, void* stream);
+
+/*
+ * b200attn_quantize_workspace_bytes -- device workspace b200attn_quantize_fp8
+ * needs for these sizes: B*H*ceil(N/128)*4 bytes for SCALE_PER_HEAD (one
+ * partial absmax per 128-token block), 0 for SCALE_PER_BLOCK. Returns 0 for
+ * invalid sizes.
+ */
+size_t b200attn_quantize_workspace_bytes(int B, int N, int H, int d, int granularity);
+
+/*
+ * b200attn_quantize_fp8 -- absmax quantisation of a bf16 tensor to e4m3, with
+ * an optional orthonormal Hadamard rotation along d applied first.
+ *
+ * Defined by: "Zyphra ZYFA: 1.76x …", "ZYFA's performance and accuracy data"
+ * (E4M3 with per-tensor or per-head scale factors that map values into the
+ * representable range) and "Zyphra 开源 ZYFA …", "ZYFA 的 FP8 注意力有多准确？"
+ * (a Hadamard rotation of Q and K roughly halves the input-quantisation error).
+ *
+ * Per scale group g (a head, or a 128-token block of a head), in fp32:
+ *   y      = x                                   (hadamard == 0)
+ *          = H_128 x / sqrt(128)                 (hadamard == 1, d == 128)
+ *          = (H_128 (+) H_64) x, scaled by 1/sqrt(128) and 1/8 (d == 192)
+ *            with H_n the Sylvester Hadamard matrix, evaluated with radix-2
+ *            butterflies of widths 1, 2, 4, ... (lower element a+b, upper a-b)
+ *   amax   = max |y| over the group
+ *   inv    = 448 / amax,  scale = amax / 448      (both 1 when amax == 0)
+ *   code   = e4m3(y * inv), round to nearest even, saturating at +-448
+ * Codes are bit-identical for identical inputs on every call.
+ *
+ * x          [B, N, H, d] bf16 device pointer
+ * x_fp8      [B, N, H, d] e4m3 output (one byte per element)
+ * scale      fp32 output, [B, H] or [B, H, ceil(N/128)] by granularity
+ * d          128 or 192 (the head dims b200attn_fwd takes)
+ * hadamard   0 or 1 (apply to Q and K only; V is quantised unrotated)
+ * workspace  device scratch of at least b200attn_quantize_workspace_bytes
+ *            bytes (may be NULL when that is 0); owned by the caller, its
+ *            contents on entry do not matter, and concurrent calls must use
+ *            distinct workspaces
+ *
+ * Errors: INVALID, UNSUPPORTED (d not 128/192), WORKSPACE, CUDA.
+ */
+int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale,
+                          int B, int N, int H, int d,
+                          int granularity, int hadamard,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * b200attn_check -- synchronise `stream`, then return and clear the device
+ * status word: 0, or B200ATTN_ERR_TIMEOUT if any kernel of this library gave
+ * up on a wait since the last check; B200ATTN_ERR_CUDA if synchronising fails.
+ */
+int b200attn_check(void* stream);
+
+/* Static description of a status code; never NULL. */
+const char* b200attn_strerror(int code);
+
+/* B200ATTN_VERSION of the built library. */
+int b200attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* B200ATTN_H_ */

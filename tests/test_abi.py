@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and loads,
+exports every entry point include/b200attn.h declares, and rejects bad
+arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "b200attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bf16_causal_prefill_fwd_b200 import build
+    build.build()
+    from bf16_causal_prefill_fwd_b200 import _binding
+    return _binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(b200attn_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("b200attn_fwd", "b200attn_quantize_fp8", "b200attn_quantize_workspace_bytes",
+                 "b200attn_check", "b200attn_strerror", "b200attn_version"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from bf16_causal_prefill_fwd_b200 import LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r" T (b200attn_\w+)$", out, re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_version_and_strerror(lib):
+    text = open(HEADER).read()
+    ver = int(re.search(r"#define B200ATTN_VERSION (\d+)", text).group(1))
+    assert lib.b200attn_version() == ver
+    for code in (0, -1, -2, -3, -4, -5, 12345):
+        assert isinstance(lib.b200attn_strerror(code), bytes)
+    assert lib.b200attn_strerror(-4) != lib.b200attn_strerror(-1)
+
+
+FAKE = 0x10000  # a 16-byte aligned non-NULL value; never dereferenced on these paths
+
+
+def fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, Hq=4, Hkv=2, N=64, dqk=128, dv=128, causal=1, dtype=0,
+        qs=None, ks=None, vs=None, gran=0, scale=0.0, lse=None):
+    return lib.b200attn_fwd(q, k, v, o, B, Hq, Hkv, N, dqk, dv, causal, dtype, qs, ks, vs, gran, scale, lse, None)
+
+
+def test_fwd_rejects_bad_arguments_on_the_host(lib):
+    assert fwd(lib, q=None) == -1
+    assert fwd(lib, o=None) == -1
+    assert fwd(lib, B=0) == -1
+    assert fwd(lib, N=0) == -1
+    assert fwd(lib, Hq=3, Hkv=2) == -1
+    assert fwd(lib, causal=2) == -1
+    assert fwd(lib, q=FAKE + 8) == -1                       # misaligned
+    assert fwd(lib, lse=FAKE + 2) == -1                     # misaligned lse
+    assert fwd(lib, dtype=1) == -1                          # FP8 without scales
+    assert fwd(lib, scale=float("nan")) == -1
+
+
+def test_fwd_reports_unsupported_shapes_on_the_host(lib):
+    assert fwd(lib, dqk=64, dv=64) == -2
+    assert fwd(lib, dqk=128, dv=192) == -2
+    assert fwd(lib, dtype=7) == -2
+    assert fwd(lib, dtype=1, qs=FAKE, ks=FAKE, vs=FAKE, gran=5) == -2
+
+
+def test_quantize_workspace_size(lib):
+    assert lib.b200attn_quantize_workspace_bytes(1, 16384, 32, 128, 0) == 1 * 32 * 128 * 4
+    assert lib.b200attn_quantize_workspace_bytes(2, 300, 8, 128, 0) == 2 * 8 * 3 * 4
+    assert lib.b200attn_quantize_workspace_bytes(2, 300, 8, 128, 1) == 0
+    assert lib.b200attn_quantize_workspace_bytes(0, 300, 8, 128, 0) == 0
+
+
+def test_quantize_rejects_bad_arguments_on_the_host(lib):
+    q = lib.b200attn_quantize_fp8
+    assert q(None, FAKE, FAKE, 1, 10, 1, 128, 0, 0, FAKE, 64, None) == -1
+    assert q(FAKE, FAKE, FAKE, 1, 0, 1, 128, 0, 0, FAKE, 64, None) == -1
+    assert q(FAKE, FAKE, FAKE, 1, 10, 1, 64, 0, 0, FAKE, 64, None) == -2
+    assert q(FAKE, FAKE, FAKE, 1, 10, 1, 128, 3, 0, FAKE, 64, None) == -2
+    assert q(FAKE, FAKE, FAKE, 1, 10, 1, 128, 0, 2, FAKE, 64, None) == -1
+    assert q(FAKE + 4, FAKE, FAKE, 1, 10, 1, 128, 0, 0, FAKE, 64, None) == -1
+    assert q(FAKE, FAKE, FAKE, 1, 10, 1, 128, 0, 0, None, 0, None) == -5     # per-head needs a workspace
+    assert q(FAKE, FAKE, FAKE, 1, 300, 2, 128, 0, 0, FAKE, 8, None) == -5    # too small
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import bf16_causal_prefill_fwd_b200 as b
+    x = torch.zeros(1, 8, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        b.attn_fwd(x, x, x)
+    with pytest.raises(ValueError):
+        b.quantize_fp8(x)
+
+
+def test_package_has_no_oracle_dependency():
+    """The product path never imports the oracle (it is test infrastructure)."""
+    pkg = os.path.join(ROOT, "bf16_causal_prefill_fwd_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", text, re.M), f
+                assert "attn_oracle" not in text and "liboracle" not in text, f

@@ -1,0 +1,186 @@
+"""Parity of the CUDA attention kernels (through the C ABI) with the fp64 oracle.
+
+Tolerances are relative RMS errors against fp64 attention on the identical
+inputs: 1e-2 for BF16, 6e-2 for FP8 e4m3 (inputs quantised by the oracle's
+quantizer; the kernel receives those exact bytes and scales)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import bf16_causal_prefill_fwd_b200 as b2
+from helpers import (BF16_TOL, FP8_TOL, f32, gather_sample, oracle_fp8_inputs, oracle_on_sample,
+                     sampled_rows, to_gpu_fp8)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_bf16(q, k, v, causal=True, scale=None):
+    o, lse = b2.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, softmax_scale=scale, return_lse=True)
+    assert b2.check() == 0
+    return o, lse
+
+
+def run_fp8(codes, causal=True, scale=None):
+    q8, sq, k8, sk, v8, sv = to_gpu_fp8(codes)
+    o, lse = b2.attn_fwd(q8, k8, v8, q_scale=sq, k_scale=sk, v_scale=sv, causal=causal,
+                         softmax_scale=scale, return_lse=True)
+    assert b2.check() == 0
+    return o, lse
+
+
+SMALL = [
+    # B, Hq, Hkv, N, d_qk
+    (1, 1, 1, 256, 128),     # the tiny workload's shape
+    (1, 4, 2, 1, 128),
+    (1, 4, 2, 2, 128),
+    (1, 4, 2, 127, 128),
+    (1, 4, 2, 128, 128),
+    (1, 4, 2, 129, 128),
+    (1, 4, 2, 255, 128),
+    (1, 4, 2, 257, 128),
+    (2, 4, 1, 300, 128),
+    (1, 8, 8, 384, 128),
+    (1, 8, 1, 640, 128),
+    (3, 2, 2, 1000, 128),
+    (1, 2, 2, 1, 192),
+    (1, 4, 4, 300, 192),
+    (2, 2, 1, 700, 192),
+]
+
+
+def check_lse(lse_gpu, ref_lse):
+    got = lse_gpu.cpu().numpy().transpose(0, 2, 1)   # [B,Hq,N] -> [B,N,Hq]
+    np.testing.assert_allclose(got, ref_lse, rtol=0, atol=2e-3)
+
+
+@pytest.mark.parametrize("shape", SMALL)
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_matches_oracle(shape, causal):
+    B, Hq, Hkv, N, dqk = shape
+    q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq))
+    o, lse = run_bf16(q, k, v, causal)
+    ref, ref_lse = oracle.attention(f32(q), f32(k), f32(v), causal=causal)
+    err = oracle.rel_rms(f32(o), ref)
+    assert err <= BF16_TOL, err
+    assert np.isfinite(f32(o)).all()
+    check_lse(lse, ref_lse)
+
+
+@pytest.mark.parametrize("shape", SMALL)
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_matches_oracle(shape, causal):
+    B, Hq, Hkv, N, dqk = shape
+    q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq + 1))
+    codes, deq = oracle_fp8_inputs(q, k, v)
+    o, lse = run_fp8(codes, causal)
+    ref, ref_lse = oracle.attention(*deq, causal=causal)
+    err = oracle.rel_rms(f32(o), ref)
+    assert err <= FP8_TOL, err
+    check_lse(lse, ref_lse)
+
+
+def test_tiny_workload_both_dtypes():
+    w = workloads.tiny()
+    q, k, v = workloads.draw(w)
+    ref, _ = oracle.attention(f32(q), f32(k), f32(v))
+    o, _ = run_bf16(q, k, v)
+    e_bf16 = oracle.rel_rms(f32(o), ref)
+    codes, deq = oracle_fp8_inputs(q, k, v)
+    ref8, _ = oracle.attention(*deq)
+    o8, _ = run_fp8(codes)
+    e_fp8 = oracle.rel_rms(f32(o8), ref8)
+    e_fp8_unq = oracle.rel_rms(f32(o8), ref)
+    print(f"tiny: bf16 {e_bf16:.2e}  fp8 {e_fp8:.2e}  fp8-vs-unquantised {e_fp8_unq:.2e}")
+    assert e_bf16 <= BF16_TOL and e_fp8 <= FP8_TOL
+
+
+def test_explicit_softmax_scale():
+    q, k, v = workloads.draw(workloads.gaussian(1, 2, 1, 200, 128, 128, seed=5))
+    o, lse = run_bf16(q, k, v, scale=0.02)
+    ref, ref_lse = oracle.attention(f32(q), f32(k), f32(v), softmax_scale=0.02)
+    assert oracle.rel_rms(f32(o), ref) <= BF16_TOL
+    check_lse(lse, ref_lse)
+
+
+def test_first_row_is_v0_and_prefix_mean():
+    """Row 0 returns v_0; with Q = 0 every row is the running mean of V."""
+    q, k, v = workloads.draw(workloads.gaussian(1, 2, 2, 300, 128, 128, seed=6))
+    o, _ = run_bf16(q, k, v)
+    np.testing.assert_allclose(f32(o)[0, 0], f32(v)[0, 0], rtol=1e-2, atol=1e-2)
+    z = torch.zeros_like(q)
+    o0, _ = run_bf16(z, k, v)
+    prefix = np.cumsum(f32(v)[0].astype(np.float64), axis=0) / np.arange(1, 301)[:, None, None]
+    assert oracle.rel_rms(f32(o0)[0], prefix) <= BF16_TOL
+
+
+def test_causality_on_gpu():
+    """Changing keys/values after position i leaves rows <= i bit-identical."""
+    q, k, v = workloads.draw(workloads.gaussian(1, 4, 2, 512, 128, 128, seed=7))
+    o1, _ = run_bf16(q, k, v)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, 300:] = torch.randn_like(k2[:, 300:].float()).to(torch.bfloat16)
+    v2[:, 300:] = torch.randn_like(v2[:, 300:].float()).to(torch.bfloat16)
+    o2, _ = run_bf16(q, k2, v2)
+    assert torch.equal(o1[:, :300], o2[:, :300])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_bitwise_deterministic_over_1000_launches(dtype):
+    q, k, v = workloads.draw(workloads.gaussian(1, 8, 2, 2048, 128, 128, seed=8))
+    if dtype == "bf16":
+        args = (q.cuda(), k.cuda(), v.cuda())
+        kw = {}
+    else:
+        q8, sq, k8, sk, v8, sv = to_gpu_fp8(oracle_fp8_inputs(q, k, v)[0])
+        args = (q8, k8, v8)
+        kw = dict(q_scale=sq, k_scale=sk, v_scale=sv)
+    first = b2.attn_fwd(*args, **kw)
+    out = torch.empty_like(first)
+    same = torch.ones((), dtype=torch.bool, device="cuda")
+    for _ in range(1000):
+        b2.attn_fwd(*args, out=out, **kw)
+        same &= (out.view(torch.int16) == first.view(torch.int16)).all()
+    assert b2.check() == 0
+    assert bool(same)
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled rows
+
+FULL = {
+    "gqa7b": workloads.gqa7b,
+    "qknorm": workloads.qknorm,
+    "mla": workloads.mla,
+}
+
+
+@pytest.mark.parametrize("name", ["gqa7b", "mla"])
+def test_full_size_bf16_sampled(name):
+    w = FULL[name]()
+    q, k, v = workloads.draw(w)
+    o, _ = run_bf16(q, k, v)
+    heads = sorted({0, 1, w.Hq // w.Hkv, w.Hq - 1})
+    rows = sampled_rows(w.N)
+    ref, _ = oracle_on_sample(q, k, v, heads, rows)
+    err = oracle.rel_rms(gather_sample(o, heads, rows), ref)
+    print(f"{name} bf16 sampled rel-rms {err:.2e}")
+    assert err <= BF16_TOL
+    assert torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("qknorm", False), ("qknorm", True), ("mla", False)])
+def test_full_size_fp8_sampled(name, hadamard):
+    w = FULL[name]()
+    q, k, v = workloads.draw(w)
+    heads = sorted({0, 1, w.Hq // w.Hkv, w.Hq - 1})
+    rows = sampled_rows(w.N)
+    # quantise only what the sample needs plus the whole tensors for the GPU
+    codes, deq = oracle_fp8_inputs(q, k, v, hadamard=hadamard)
+    o, _ = run_fp8(codes)
+    ref8, _ = oracle_on_sample(*deq, heads, rows)
+    got = gather_sample(o, heads, rows)
+    err = oracle.rel_rms(got, ref8)
+    ref, _ = oracle_on_sample(q, k, v, heads, rows)
+    print(f"{name} fp8 (hadamard={hadamard}) rel-rms {err:.2e}; vs unquantised fp64 {oracle.rel_rms(got, ref):.2e}")
+    assert err <= FP8_TOL

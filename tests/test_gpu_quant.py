@@ -1,0 +1,54 @@
+"""The CUDA e4m3 quantizer (through the C ABI) against the oracle's quantizer:
+codes and scales must be bit-identical (integer work, decided in fp32 on both
+sides with the same operations)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import bf16_causal_prefill_fwd_b200 as b2
+from helpers import f32
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_quant(x, granularity, hadamard):
+    codes, scale = b2.quantize_fp8(x.cuda(), granularity=granularity, hadamard=hadamard)
+    assert b2.check() == 0
+    return codes.view(torch.uint8).cpu().numpy(), scale.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 128), (2, 300, 3, 128), (1, 129, 2, 192), (2, 1000, 1, 192),
+                                   (1, 256, 4, 128)])
+@pytest.mark.parametrize("granularity", ["head", "block"])
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_codes_and_scales_bit_exact(shape, granularity, hadamard):
+    B, N, H, d = shape
+    g = torch.Generator().manual_seed(B * 1000 + N + H + d)
+    x = (torch.randn(B, N, H, d, generator=g) * torch.exp(torch.randn(H, d, generator=g))).to(torch.bfloat16)
+    codes, scale = gpu_quant(x, granularity, hadamard)
+    ref_codes, ref_scale = oracle.quantize_fp8(f32(x), granularity, hadamard)
+    assert np.array_equal(scale, ref_scale)
+    assert np.array_equal(codes, ref_codes)
+
+
+def test_zero_and_saturation_cases():
+    x = torch.zeros(1, 130, 2, 128, dtype=torch.bfloat16)
+    x[0, 129, 1, 5] = -3.0
+    for gran in ("head", "block"):
+        codes, scale = gpu_quant(x, gran, False)
+        ref_codes, ref_scale = oracle.quantize_fp8(f32(x), gran, False)
+        assert np.array_equal(codes, ref_codes) and np.array_equal(scale, ref_scale)
+    assert codes[0, 129, 1, 5] == 0xFE  # -448
+
+
+@pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("qknorm", True)])
+def test_full_size_q_bit_exact(name, hadamard):
+    w = workloads.BY_NAME[name]()
+    q, k, v = workloads.draw(w)
+    for t, rot in ((k, hadamard), (v, False)):
+        codes, scale = gpu_quant(t, "head", rot)
+        ref_codes, ref_scale = oracle.quantize_fp8(f32(t), "head", rot)
+        assert np.array_equal(scale, ref_scale)
+        assert np.array_equal(codes, ref_codes)
