@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Causal prefill attention benchmark on B200: TFLOP/s of one step of the hot path.
+
+A step is one pass of the whole path over one layer of synthetic input:
+  FP8 (default): e4m3 quantizer on Q, K and V (per-head scales), then the FP8
+                 attention kernel;
+  BF16:          the BF16 attention kernel.
+Default workload: the 7B-style GQA layer, B=1, Hq=32, Hkv=8, N=16384,
+d_qk=d_v=128, causal. FLOPs use the FlashAttention convention
+B*Hq*N^2*(d_qk+d_v) (the causal half of the two matmuls).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--dtype fp8|bf16]
+                    [--workload gqa7b|qknorm|mla|sweepN] [--n N] [--impl ours|reference]
+
+N > 1 runs as one process per GPU under torch.distributed.run; every rank
+runs its own replica of the layer (the path has no exchange step), and rank 0
+prints one JSON line with the whole-job throughput (max time over ranks).
+``--impl reference`` times the CPU fp64 oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "causal prefill attn TFLOP/s (FP8 e4m3, BF16) at 16K/32K; % of B200 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--dtype", choices=["fp8", "bf16"], default="fp8")
+    ap.add_argument("--workload", default="gqa7b")
+    ap.add_argument("--n", type=int, default=None, help="sequence length override")
+    ap.add_argument("--hadamard", action="store_true", help="rotate Q and K before FP8 quantisation")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-dtype", action="store_true", help="skip the secondary dtype measurement")
+    return ap.parse_args()
+
+
+def make_workload(name: str, n: int | None) -> workloads.Workload:
+    if name.startswith("sweep"):
+        return workloads.sweep(int(name[5:]) if len(name) > 5 else (n or 16384))
+    fn = workloads.BY_NAME[name]
+    return fn(n) if n and name != "tiny" else fn()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_fwd_kernel.cuh", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "bf16_causal_prefill_fwd_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key: str, workload_name: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the
+    current kernel source; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel_key, {}).get(workload_name)
+    if not e or e.get("src_sha") != kernel_sources_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                pw.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "power_w_max": max(pw),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# reference arm / CPU baseline: the fp64 oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------------------------
+
+def oracle_sample(q, k, v, w: workloads.Workload, target_s: float, max_rows: int | None = None):
+    """Time the fp64 oracle on rows of query head 0 (batch 0), rows spread over the sequence,
+    growing the sample until it has taken about target_s. Returns (TFLOP/s, desc, seconds)."""
+    import oracle
+    G = w.Hq // w.Hkv
+    qs = q[0:1, :, 0:1].float().numpy().astype(np.float64)
+    ks = k[0:1, :, 0:1].float().numpy().astype(np.float64)
+    vs = v[0:1, :, 0:1].float().numpy().astype(np.float64)
+    _ = G
+    rng = np.random.default_rng(0)
+    n_rows, flops, secs = 64, 0.0, 0.0
+    done_rows = 0
+    while True:
+        rows = np.sort(rng.integers(0, w.N, n_rows))
+        trip = np.stack([np.zeros_like(rows), np.zeros_like(rows), rows], axis=1).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention(qs, ks, vs, causal=True, rows=trip)
+        secs += time.perf_counter() - t0
+        flops += float(np.sum(rows + 1)) * 2.0 * (w.d_qk + w.d_v)
+        done_rows += n_rows
+        if secs >= target_s or (max_rows and done_rows >= max_rows):
+            break
+        n_rows = min(n_rows * 2, 1 << 16)
+    desc = (f"{done_rows} query rows of head 0 (batch 0) spread uniformly over N={w.N}, causal, "
+            f"fp64; FLOPs counted as 2*(i+1)*(d_qk+d_v) per row i")
+    return flops / secs / 1e12, desc, secs
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    w = make_workload(args.workload, args.n)
+    q, k, v = workloads.draw(w)
+    cores = len(os.sched_getaffinity(0))
+    per_step = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        tf, desc, secs = oracle_sample(q, k, v, w, target_s=0.5)
+        if i >= args.warmup:
+            per_step.append(tf)
+    val = statistics.median(per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name} B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d_qk={w.d_qk} d_v={w.d_v} causal",
+                   "sample": desc},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+class Path:
+    """Preallocated buffers and the step of the hot path for one dtype."""
+
+    def __init__(self, b2, q, k, v, dtype: str, hadamard: bool):
+        self.b2, self.q, self.k, self.v, self.dtype, self.hadamard = b2, q, k, v, dtype, hadamard
+        B, N, Hq, dqk = q.shape
+        Hkv, dv = k.shape[2], v.shape[3]
+        dev = q.device
+        self.o = torch.empty((B, N, Hq, dv), dtype=torch.bfloat16, device=dev)
+        if dtype == "fp8":
+            self.q8 = torch.empty(q.shape, dtype=torch.float8_e4m3fn, device=dev)
+            self.k8 = torch.empty(k.shape, dtype=torch.float8_e4m3fn, device=dev)
+            self.v8 = torch.empty(v.shape, dtype=torch.float8_e4m3fn, device=dev)
+            self.sq = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+            self.sk = torch.empty((B, Hkv), dtype=torch.float32, device=dev)
+            self.sv = torch.empty((B, Hkv), dtype=torch.float32, device=dev)
+            ws = max(b2.quantize_workspace_bytes(B, N, Hq, dqk), 4)
+            self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.launches_per_step = 7 if dtype == "fp8" else 1
+
+    def step(self, ev_a0=None, ev_a1=None):
+        b2 = self.b2
+        if self.dtype == "fp8":
+            b2.quantize_fp8(self.q, hadamard=self.hadamard, out=self.q8, scale=self.sq, workspace=self.ws)
+            b2.quantize_fp8(self.k, hadamard=self.hadamard, out=self.k8, scale=self.sk, workspace=self.ws)
+            b2.quantize_fp8(self.v, hadamard=False, out=self.v8, scale=self.sv, workspace=self.ws)
+            if ev_a0 is not None:
+                ev_a0.record()
+            b2.attn_fwd(self.q8, self.k8, self.v8, q_scale=self.sq, k_scale=self.sk, v_scale=self.sv,
+                        out=self.o)
+        else:
+            if ev_a0 is not None:
+                ev_a0.record()
+            b2.attn_fwd(self.q, self.k, self.v, out=self.o)
+        if ev_a1 is not None:
+            ev_a1.record()
+
+
+def time_path(path: Path, steps: int, warmup: int, flush, dist_on: bool):
+    for _ in range(warmup):
+        path.step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for e0, e1, a0, a1 in evs:
+        flush.zero_()  # L2 flush, outside the step's events
+        e0.record()
+        path.step(a0, a1)
+        e1.record()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    step_ms = [e0.elapsed_time(e1) for e0, e1, _, _ in evs]
+    attn_ms = [a0.elapsed_time(a1) for _, _, a0, a1 in evs]
+    return step_ms, attn_ms
+
+
+def max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import bf16_causal_prefill_fwd_b200 as b2
+    b2.load_library()
+    dist_on = world > 1
+    torch.cuda.set_device(local_rank)
+    w = make_workload(args.workload, args.n)
+    q_cpu, k_cpu, v_cpu = workloads.draw(w)
+    q, k, v = q_cpu.cuda(), k_cpu.cuda(), v_cpu.cuda()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    peaks, peak_src = load_peaks()
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+
+    def measure(dtype):
+        path = Path(b2, q, k, v, dtype, args.hadamard)
+        step_ms, attn_ms = time_path(path, args.steps, args.warmup, flush, dist_on)
+        if b2.check() != 0:
+            raise RuntimeError("a kernel reported a timeout")
+        ms = max_over_ranks(statistics.mean(step_ms), dist_on)
+        ams = max_over_ranks(statistics.mean(attn_ms), dist_on)
+        value = world * w.flops / (ms * 1e-3) / 1e12
+        achieved = w.flops / (ams * 1e-3) / 1e12
+        peak = bf16_peak * (2.0 if dtype == "fp8" else 1.0)
+        kernel_key = f"attn_fwd_kernel<{w.d_qk},{w.d_v},{'fp8' if dtype == 'fp8' else 'bf16'}>"
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic_for(kernel_key, w.name),
+                "kernel": kernel_key, "kernel_ms": ams,
+                "peak_source": (f"{peak_src} bf16 burst {bf16_peak} TFLOP/s"
+                                + (" x2 (nominal fp8/bf16 ratio 4.5/2.25)" if dtype == "fp8" else "")),
+                "frac_of_spec_dense": achieved / (4500.0 if dtype == "fp8" else 2250.0)}
+        return {"value": value, "ms_per_step": ms, "roofline": roof,
+                "launches": path.launches_per_step * args.steps,
+                "step_ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))]}
+
+    with ClockSampler(local_rank) as clk:
+        main = measure(args.dtype)
+    clocks = clk.summary()
+    other = None
+    if not args.no_other_dtype:
+        other_dtype = "bf16" if args.dtype == "fp8" else "fp8"
+        other = measure(other_dtype)
+        other["dtype"] = other_dtype
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(b2, args, w, q_cpu, k_cpu, v_cpu, world, dist_on)
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        tf, desc, secs = oracle_sample(q_cpu, k_cpu, v_cpu, w, target_s=10.0)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": desc, "seconds": secs}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": main["value"], "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3" if args.dtype == "fp8" else "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d_qk={w.d_qk} "
+                                   f"d_v={w.d_v} causal, seed {w.seed}",
+                       "step": ("e4m3 quantizer on Q,K,V (per-head scales"
+                                + (", Hadamard on Q,K" if args.hadamard else "") + ") + FP8 attention")
+                       if args.dtype == "fp8" else "BF16 attention",
+                       "flops_per_step": w.flops, "flop_convention": "B*Hq*N^2*(d_qk+d_v)",
+                       "l2": "256 MiB buffer written between timed steps (untimed); inputs exceed L2",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": main["roofline"],
+            "clocks": clocks,
+            "gpu_launches": main["launches"],
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "step_ms_p10_p90": main["step_ms_p10_p90"],
+        }
+        if other is not None:
+            line["other_dtype"] = other
+        print(json.dumps(line), flush=True)
+
+
+def measure_e2e(b2, args, w, q_cpu, k_cpu, v_cpu, world, dist_on):
+    """Same metric through the public API from pinned host buffers: H2D of Q,K,V, the
+    step (quantizer + attention), D2H of O, all inside the timed region."""
+    hq, hk, hv = q_cpu.pin_memory(), k_cpu.pin_memory(), v_cpu.pin_memory()
+    ho = torch.empty((w.B, w.N, w.Hq, w.d_v), dtype=torch.bfloat16).pin_memory()
+    q = torch.empty_like(q_cpu, device="cuda")
+    k = torch.empty_like(k_cpu, device="cuda")
+    v = torch.empty_like(v_cpu, device="cuda")
+    path = Path(b2, q, k, v, args.dtype, args.hadamard)
+
+    def step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        path.step()
+        ho.copy_(path.o, non_blocking=True)
+
+    steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist_on)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
+    return {"value": world * w.flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
