@@ -47,13 +47,17 @@ L2_FLUSH_BYTES = 256 << 20
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--dtype", choices=["fp8", "bf16"], default="fp8")
     ap.add_argument("--workload", default="gqa7b")
     ap.add_argument("--n", type=int, default=None, help="sequence length override")
     ap.add_argument("--hadamard", action="store_true", help="rotate Q and K before FP8 quantisation")
+    ap.add_argument("--fp8-p", choices=["lean", "mufu"], default=None,
+                    help="how the FP8 kernel forms probabilities (default: the library default, Lean P)")
+    ap.add_argument("--settle-s", type=float, default=1.0,
+                    help="untimed back-to-back steps before timing so clocks reach their sustained level")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-dtype", action="store_true", help="skip the secondary dtype measurement")
@@ -101,60 +105,71 @@ def traffic_for(kernel_key: str, workload_name: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clock, power and clock-event reasons sampled every 10 ms through NVML in a thread;
+    summary() reports the samples that fall inside the marked timed window."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device: int, interval_s: float = 0.01):
+        self.samples = []
+        self.window = []
+        self.interval = interval_s
+        self._stop = threading.Event()
+        self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:  # noqa: BLE001
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(props.uuid)).encode())
+            self.nv = pynvml
+        except Exception:  # noqa: BLE001 - no NVML: report no clocks
+            self.handle = None
+
+    def _loop(self):
+        nv, h = self.nv, self.handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.interval)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+        if self.handle is not None:
+            self.thread = threading.Thread(target=self._loop, daemon=True)
             self.thread.start()
-        except OSError:
-            self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def mark(self):
+        self.window.append(time.perf_counter())
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self.handle is not None:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, pw, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-                pw.append(float(parts[3]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "power_w_max": max(pw),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.handle is None or len(self.window) < 2:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "unavailable"}
+        t0, t1 = self.window[0], self.window[-1]
+        sel = [x for x in self.samples if t0 <= x[0] <= t1] or self.samples[-3:]
+        reasons = set()
+        for x in sel:
+            for bit, name in self.REASONS.items():
+                if x[4] & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x[1] for x in sel), "sm_max_mhz": max(x[2] for x in sel),
+                "power_w_max": max(x[3] for x in sel), "reasons": sorted(reasons), "samples": len(sel),
+                "source": "nvml every 10 ms inside the timed window"}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -256,21 +271,30 @@ class Path:
             ev_a1.record()
 
 
-def time_path(path: Path, steps: int, warmup: int, flush, dist_on: bool):
+def time_path(path: Path, steps: int, warmup: int, settle_s: float, flush, dist_on: bool, clk=None):
     for _ in range(warmup):
         path.step()
     torch.cuda.synchronize()
+    t_end = time.perf_counter() + settle_s
+    while time.perf_counter() < t_end:
+        for _ in range(10):
+            path.step()
+        torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
             torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    if clk is not None:
+        clk.mark()
     for e0, e1, a0, a1 in evs:
         flush.zero_()  # L2 flush, outside the step's events
         e0.record()
         path.step(a0, a1)
         e1.record()
     torch.cuda.synchronize()
+    if clk is not None:
+        clk.mark()
     if dist_on:
         torch.distributed.barrier()
     step_ms = [e0.elapsed_time(e1) for e0, e1, _, _ in evs]
@@ -298,9 +322,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peaks, peak_src = load_peaks()
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
 
-    def measure(dtype):
+    def measure(dtype, clk=None):
         path = Path(b2, q, k, v, dtype, args.hadamard)
-        step_ms, attn_ms = time_path(path, args.steps, args.warmup, flush, dist_on)
+        step_ms, attn_ms = time_path(path, args.steps, args.warmup, args.settle_s, flush, dist_on, clk)
         if b2.check() != 0:
             raise RuntimeError("a kernel reported a timeout")
         ms = max_over_ranks(statistics.mean(step_ms), dist_on)
@@ -320,7 +344,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "step_ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))]}
 
     with ClockSampler(local_rank) as clk:
-        main = measure(args.dtype)
+        main = measure(args.dtype, clk)
     clocks = clk.summary()
     other = None
     if not args.no_other_dtype:
@@ -351,6 +375,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                        if args.dtype == "fp8" else "BF16 attention",
                        "flops_per_step": w.flops, "flop_convention": "B*Hq*N^2*(d_qk+d_v)",
                        "l2": "256 MiB buffer written between timed steps (untimed); inputs exceed L2",
+                       "settle": f"{args.settle_s} s of untimed back-to-back steps before timing",
+                       "fp8_p": os.environ.get("B200ATTN_FP8_P", "lean") if args.dtype == "fp8" else None,
                        "parallelism": f"replicas x{world}"},
             "roofline": main["roofline"],
             "clocks": clocks,
@@ -404,6 +430,8 @@ def main():
     args = parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.fp8_p:
+        os.environ["B200ATTN_FP8_P"] = args.fp8_p
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

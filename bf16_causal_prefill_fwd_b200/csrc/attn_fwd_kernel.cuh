@@ -43,6 +43,21 @@
 // T lets the running max lag the true one (P <= 2^(T+E)), which skips most O
 // rescales; E shifts FP8 probabilities up so the e4m3 normal range covers more
 // binades. Both cancel exactly in O_acc / l.
+//
+// FP8 probabilities, two ways (a template switch, chosen on the host):
+//  * MUFU: P = e4m3(ex2(x)), round to nearest even.
+//  * Lean P ("ZYFA 如何工作？", Lean P：用一次乘加代替指数运算): read as an
+//    integer, the e4m3 code of 2^x is close to 8x + 56 (+8 per doubling), so the
+//    code is built with fused multiply-adds and no exponential: one saturating
+//    FFMA gives w = clamp((8x + 56)/126, 0, 1), a pack to f16x2 and one f16x2
+//    FMA with the magic 1536 (f16 spacing 1 in [1024, 2048)) leave
+//    round(126 w) in the low byte of each lane, and one PRMT gathers four codes.
+// Either way l is the sum of the rounded probabilities the PV MMA multiplies
+// ("逐块缩放与舍入行和": divide by the sum of the rounded probabilities): the
+// bits (code << 7) read as an f16 are exactly decode(code) / 256 for every
+// non-negative e4m3 code (subnormals and zero included), so two codes are
+// decoded by one integer multiply-add and summed by one f16x2 add; each
+// block's f16 partial sums are widened to fp32.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -74,7 +89,7 @@ struct AttnParams {
   float* lse;
 };
 
-template <int DQK, int DV, bool FP8>
+template <int DQK, int DV, bool FP8, bool LEANP = false>
 struct AttnCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int CHUNK_ELEMS = 128 / ESZ;  // elements in one 128-byte swizzled row
@@ -93,7 +108,8 @@ struct AttnCfg {
   // P columns: bf16 packs 2 keys per 32-bit column, e4m3 packs 4.
   static constexpr int P_COLS = kBN * ESZ / 4;
   static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
-  static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2)
+  static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
+  static_assert(!LEANP || FP8, "Lean P builds e4m3 codes");
   static constexpr uint32_t IDESC_QK = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, kBN, false);
   static constexpr uint32_t IDESC_PV = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DV, true);
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
@@ -133,7 +149,7 @@ __device__ __forceinline__ int unit_for(int k, int cta, int grid) {
 
 // Bounded mbarrier wait. Returns false if it gave up (2 s) or another role
 // already gave up; the first to give up records the timeout status.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
@@ -153,11 +169,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort_flag);
 }
 
-template <int DQK, int DV, bool FP8>
+template <int DQK, int DV, bool FP8, bool LEANP>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<DQK, DV, FP8>;
+  using C = AttnCfg<DQK, DV, FP8, LEANP>;
   extern __shared__ uint8_t smem_raw[];
 
   // 1024-byte aligned base (128-byte swizzle atoms repeat every 1024 bytes).
@@ -445,16 +461,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
 
+        // row max: four independent three-input max chains
         float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
         float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-          mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-          mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+        for (int c = 4; c < 124; c += 8) {
+          mx0 = max3f(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+          mx1 = max3f(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+          mx2 = max3f(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+          mx3 = max3f(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        mx0 = max3f(mx0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
+        mx1 = max3f(mx1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
+        const float mx = max3f(mx0, mx1, fmaxf(mx2, mx3));
         const float m_new = fmaxf(m_run, mx * c_log2);
         const bool need = m_new > m_run + C::T_LAG;
         float alpha = 1.0f;
@@ -465,9 +484,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l_run *= alpha;
 
         // probabilities, packed in place (entry c/2 or c/4 is already consumed)
-        const float nm = C::E_SHIFT - m_run;
-        float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float l_blk;
         if constexpr (!FP8) {
+          const float nm = C::E_SHIFT - m_run;
+          float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 128; c += 2) {
             const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, nm));
@@ -477,21 +497,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_st32(tS + 0, sr);
           tmem_st32(tS + 32, sr + 32);
+          l_blk = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
         } else {
+          // acc: f16x2 partial sums of decode(code)/256 (8 adds per accumulator per block)
+          uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          if constexpr (LEANP) {
+            // w = clamp((8 (c*S - m_run + E) + 56) / 126, 0, 1); code = round(126 w)
+            const float A = c_log2 * (8.0f / 126.0f);
+            const float Bc = (8.0f * (C::E_SHIFT - m_run) + 56.0f) * (1.0f / 126.0f);
 #pragma unroll
-          for (int c = 0; c < 128; c += 4) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, nm));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), c_log2, nm));
-            const float p2 = ex2_approx(fmaf(__uint_as_float(sr[c + 2]), c_log2, nm));
-            const float p3 = ex2_approx(fmaf(__uint_as_float(sr[c + 3]), c_log2, nm));
-            sum[(c >> 2) & 7] += (p0 + p1) + (p2 + p3);
-            const uint32_t lo = pack_e4m3x2(p0, p1);
-            const uint32_t hi = pack_e4m3x2(p2, p3);
-            sr[c >> 2] = lo | (hi << 16);
+            for (int c = 0; c < 128; c += 4) {
+              const float w0 = fma_sat(__uint_as_float(sr[c]), A, Bc);
+              const float w1 = fma_sat(__uint_as_float(sr[c + 1]), A, Bc);
+              const float w2 = fma_sat(__uint_as_float(sr[c + 2]), A, Bc);
+              const float w3 = fma_sat(__uint_as_float(sr[c + 3]), A, Bc);
+              // f16 lanes 1536 + code: bits 0x6600 + code
+              const uint32_t u01 = hfma2(pack_f16x2(w0, w1), 0x57E057E0u /*126*/, 0x66006600u /*1536*/);
+              const uint32_t u23 = hfma2(pack_f16x2(w2, w3), 0x57E057E0u, 0x66006600u);
+              const int jj = (c >> 1) & 7;
+              // (u - 0x66006600) * 128: each lane becomes code << 7
+              acc[jj] = hadd2(acc[jj], u01 * 128u + 0xFFCD0000u);
+              acc[jj + 1] = hadd2(acc[jj + 1], u23 * 128u + 0xFFCD0000u);
+              sr[c >> 2] = prmt(u01, u23, 0x6420u);  // bytes: code0, code1, code2, code3
+            }
+          } else {
+            const float nm = C::E_SHIFT - m_run;
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, nm));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), c_log2, nm));
+              const float p2 = ex2_approx(fmaf(__uint_as_float(sr[c + 2]), c_log2, nm));
+              const float p3 = ex2_approx(fmaf(__uint_as_float(sr[c + 3]), c_log2, nm));
+              const uint32_t w = static_cast<uint32_t>(pack_e4m3x2(p0, p1)) |
+                                 (static_cast<uint32_t>(pack_e4m3x2(p2, p3)) << 16);
+              const int jj = (c >> 1) & 7;
+              acc[jj] = hadd2(acc[jj], prmt(w, 0u, 0x4140u) * 128u);  // code0 << 7 | code1 << 23
+              acc[jj + 1] = hadd2(acc[jj + 1], prmt(w, 0u, 0x4342u) * 128u);
+              sr[c >> 2] = w;
+            }
           }
           tmem_st32(tS + 0, sr);
+          const float s01 = f16x2_sum_f32(acc[0]) + f16x2_sum_f32(acc[1]);
+          const float s23 = f16x2_sum_f32(acc[2]) + f16x2_sum_f32(acc[3]);
+          const float s45 = f16x2_sum_f32(acc[4]) + f16x2_sum_f32(acc[5]);
+          const float s67 = f16x2_sum_f32(acc[6]) + f16x2_sum_f32(acc[7]);
+          l_blk = ((s01 + s23) + (s45 + s67)) * 256.0f;
         }
-        l_run += ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+        l_run += l_blk;
 
         // rescale this tile's O accumulator (PV_t,i-1 has completed: its commit preceded S_t,i)
         if (i > 0 && __any_sync(0xffffffffu, need)) {

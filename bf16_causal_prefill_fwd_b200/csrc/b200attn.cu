@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -55,6 +56,14 @@ bool make_tmap(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, int N, i
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// How the FP8 kernel forms e4m3 probabilities: Lean P (FMA bit construction,
+// the default) or the MUFU exponential. B200ATTN_FP8_P=mufu selects the latter;
+// read on every call so A/B runs need no rebuild.
+bool fp8_lean_p() {
+  const char* e = std::getenv("B200ATTN_FP8_P");
+  return !(e && std::strcmp(e, "mufu") == 0);
+}
+
 int device_ok(int* sm_count) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return B200ATTN_ERR_CUDA;
@@ -67,15 +76,15 @@ int device_ok(int* sm_count) {
   return B200ATTN_OK;
 }
 
-template <int DQK, int DV, bool FP8>
+template <int DQK, int DV, bool FP8, bool LEANP = false>
 int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
-  using C = AttnCfg<DQK, DV, FP8>;
+  using C = AttnCfg<DQK, DV, FP8, LEANP>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, FP8, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, FP8, d_qk, p.Hkv, p.N, p.B) ||
       !make_tmap(&tv, v, FP8, d_v, p.Hkv, p.N, p.B))
     return B200ATTN_ERR_CUDA;
-  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8>;
+  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, LEANP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
@@ -152,8 +161,12 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
     if (d_qk == 128) return launch_attn<128, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn<192, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
   }
-  if (d_qk == 128) return launch_attn<128, 128, true>(q, k, v, p, d_qk, d_v, sm_count, st);
-  return launch_attn<192, 128, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+  if (fp8_lean_p()) {
+    if (d_qk == 128) return launch_attn<128, 128, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+    return launch_attn<192, 128, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+  }
+  if (d_qk == 128) return launch_attn<128, 128, true, false>(q, k, v, p, d_qk, d_v, sm_count, st);
+  return launch_attn<192, 128, true, false>(q, k, v, p, d_qk, d_v, sm_count, st);
 }
 
 size_t b200attn_quantize_workspace_bytes(int B, int N, int H, int d, int granularity) {

@@ -3,6 +3,8 @@
 Tolerances are relative RMS errors against fp64 attention on the identical
 inputs: 1e-2 for BF16, 6e-2 for FP8 e4m3 (inputs quantised by the oracle's
 quantizer; the kernel receives those exact bytes and scales)."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -50,9 +52,34 @@ SMALL = [
 ]
 
 
-def check_lse(lse_gpu, ref_lse):
+# The FP8 kernel forms e4m3 probabilities either with the MUFU exponential or
+# with Lean P (FMA bit construction); both are tested.
+FP8_P = ["lean", "mufu"]
+
+
+@pytest.fixture
+def fp8_p(request):
+    old = os.environ.get("B200ATTN_FP8_P")
+    os.environ["B200ATTN_FP8_P"] = request.param
+    yield request.param
+    if old is None:
+        os.environ.pop("B200ATTN_FP8_P", None)
+    else:
+        os.environ["B200ATTN_FP8_P"] = old
+
+
+def check_lse(lse_gpu, ref_lse, atol=2e-3):
     got = lse_gpu.cpu().numpy().transpose(0, 2, 1)   # [B,Hq,N] -> [B,N,Hq]
-    np.testing.assert_allclose(got, ref_lse, rtol=0, atol=2e-3)
+    np.testing.assert_allclose(got, ref_lse, rtol=0, atol=atol)
+
+
+# The FP8 kernel's lse is the log of the normaliser it actually divides by, the
+# sum of the e4m3-rounded probabilities. Rounding to e4m3 moves each normal
+# probability by at most a factor (1 +- 2^-4), so |lse - exact| <= ln(1 + 2^-4)
+# = 0.0606. Lean P also replaces 2^f by 1 + f inside each binade (at most a
+# factor 1.0615 high), so its bound is ln(1.0625 * 1.0615) = 0.1203.
+MUFU_LSE_ATOL = 0.061
+LEAN_LSE_ATOL = 0.121
 
 
 @pytest.mark.parametrize("shape", SMALL)
@@ -68,9 +95,10 @@ def test_bf16_matches_oracle(shape, causal):
     check_lse(lse, ref_lse)
 
 
+@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
 @pytest.mark.parametrize("shape", SMALL)
 @pytest.mark.parametrize("causal", [True, False])
-def test_fp8_matches_oracle(shape, causal):
+def test_fp8_matches_oracle(shape, causal, fp8_p):
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq + 1))
     codes, deq = oracle_fp8_inputs(q, k, v)
@@ -78,10 +106,11 @@ def test_fp8_matches_oracle(shape, causal):
     ref, ref_lse = oracle.attention(*deq, causal=causal)
     err = oracle.rel_rms(f32(o), ref)
     assert err <= FP8_TOL, err
-    check_lse(lse, ref_lse)
+    check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
 
 
-def test_tiny_workload_both_dtypes():
+@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
+def test_tiny_workload_both_dtypes(fp8_p):
     w = workloads.tiny()
     q, k, v = workloads.draw(w)
     ref, _ = oracle.attention(f32(q), f32(k), f32(v))
@@ -92,7 +121,7 @@ def test_tiny_workload_both_dtypes():
     o8, _ = run_fp8(codes)
     e_fp8 = oracle.rel_rms(f32(o8), ref8)
     e_fp8_unq = oracle.rel_rms(f32(o8), ref)
-    print(f"tiny: bf16 {e_bf16:.2e}  fp8 {e_fp8:.2e}  fp8-vs-unquantised {e_fp8_unq:.2e}")
+    print(f"tiny: bf16 {e_bf16:.2e}  fp8[{fp8_p}] {e_fp8:.2e}  fp8-vs-unquantised {e_fp8_unq:.2e}")
     assert e_bf16 <= BF16_TOL and e_fp8 <= FP8_TOL
 
 
@@ -126,8 +155,10 @@ def test_causality_on_gpu():
     assert torch.equal(o1[:, :300], o2[:, :300])
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
-def test_bitwise_deterministic_over_1000_launches(dtype):
+@pytest.mark.parametrize("dtype", ["bf16", "fp8-lean", "fp8-mufu"])
+def test_bitwise_deterministic_over_1000_launches(dtype, monkeypatch):
+    if dtype.startswith("fp8"):
+        monkeypatch.setenv("B200ATTN_FP8_P", dtype[4:])
     q, k, v = workloads.draw(workloads.gaussian(1, 8, 2, 2048, 128, 128, seed=8))
     if dtype == "bf16":
         args = (q.cuda(), k.cuda(), v.cuda())
@@ -169,18 +200,22 @@ def test_full_size_bf16_sampled(name):
     assert torch.isfinite(o.float()).all()
 
 
-@pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("qknorm", False), ("qknorm", True), ("mla", False)])
-def test_full_size_fp8_sampled(name, hadamard):
+@pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("gqa7b", True), ("qknorm", False), ("qknorm", True),
+                                           ("mla", False)])
+def test_full_size_fp8_sampled(name, hadamard, monkeypatch):
+    """Both ways of forming P, on the oracle's codes of the full layer; rows sampled."""
     w = FULL[name]()
     q, k, v = workloads.draw(w)
     heads = sorted({0, 1, w.Hq // w.Hkv, w.Hq - 1})
     rows = sampled_rows(w.N)
-    # quantise only what the sample needs plus the whole tensors for the GPU
     codes, deq = oracle_fp8_inputs(q, k, v, hadamard=hadamard)
-    o, _ = run_fp8(codes)
     ref8, _ = oracle_on_sample(*deq, heads, rows)
-    got = gather_sample(o, heads, rows)
-    err = oracle.rel_rms(got, ref8)
     ref, _ = oracle_on_sample(q, k, v, heads, rows)
-    print(f"{name} fp8 (hadamard={hadamard}) rel-rms {err:.2e}; vs unquantised fp64 {oracle.rel_rms(got, ref):.2e}")
-    assert err <= FP8_TOL
+    for mode in FP8_P:
+        monkeypatch.setenv("B200ATTN_FP8_P", mode)
+        o, _ = run_fp8(codes)
+        got = gather_sample(o, heads, rows)
+        err = oracle.rel_rms(got, ref8)
+        print(f"{name} fp8[{mode}] (hadamard={hadamard}) rel-rms {err:.2e}; "
+              f"vs unquantised fp64 {oracle.rel_rms(got, ref):.2e}")
+        assert err <= FP8_TOL
