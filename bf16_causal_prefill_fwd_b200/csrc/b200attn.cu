@@ -201,6 +201,60 @@ int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale, int B, int N
                   : launch_quant<192, false>(x, x_fp8, scale, B, N, H, granularity, workspace, st);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Per-head quantizer without any allocation: the partial-absmax scratch lives in
+// a static device array instead of a caller workspace.
+// ---------------------------------------------------------------------------------------------
+
+// Capacity of the static scratch, in partial-absmax slots (one float per 128-token block of
+// each (b, h)). Every device that loads this library holds it (256 KiB) until the process exits.
+static constexpr int kStaticScratchSlots = 65536;
+static __device__ __align__(256) float g_quant_scratch[kStaticScratchSlots];
+
+namespace {
+constexpr int kMaxDevices = 64;
+float* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of g_quant_scratch on the current device, looked up once per device.
+int static_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return B200ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_quant_scratch) != cudaSuccess || ptr == nullptr) return B200ATTN_ERR_CUDA;
+    g_scratch_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return B200ATTN_OK;
+}
+}  // namespace
+
+int b200attn_quantize_fp8_static(const void* x, void* x_fp8, float* scale, int B, int N, int H, int d,
+                                 int hadamard, void* stream) {
+  if (!x || !x_fp8 || !scale) return B200ATTN_ERR_INVALID;
+  if (B < 1 || N < 1 || H < 1 || d < 1) return B200ATTN_ERR_INVALID;
+  if (hadamard != 0 && hadamard != 1) return B200ATTN_ERR_INVALID;
+  if (d != 128 && d != 192) return B200ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(x_fp8) || (reinterpret_cast<uintptr_t>(scale) & 3u)) return B200ATTN_ERR_INVALID;
+  if (H > 65535 || B > 65535) return B200ATTN_ERR_UNSUPPORTED;
+  const int64_t nblk = (static_cast<int64_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  if (static_cast<int64_t>(B) * H * nblk > kStaticScratchSlots) return B200ATTN_ERR_WORKSPACE;
+  int sm_count = 0;
+  const int dev_rc = device_ok(&sm_count);
+  if (dev_rc != B200ATTN_OK) return dev_rc;
+  float* scratch = nullptr;
+  const int rc = static_scratch(&scratch);
+  if (rc != B200ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return hadamard ? launch_quant<128, true>(x, x_fp8, scale, B, N, H, B200ATTN_SCALE_PER_HEAD, scratch, st)
+                    : launch_quant<128, false>(x, x_fp8, scale, B, N, H, B200ATTN_SCALE_PER_HEAD, scratch, st);
+  return hadamard ? launch_quant<192, true>(x, x_fp8, scale, B, N, H, B200ATTN_SCALE_PER_HEAD, scratch, st)
+                  : launch_quant<192, false>(x, x_fp8, scale, B, N, H, B200ATTN_SCALE_PER_HEAD, scratch, st);
+}
+
 int b200attn_check(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return B200ATTN_ERR_CUDA;
   int status = 0;

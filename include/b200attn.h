@@ -30,7 +30,8 @@
  *   seconds); if one runs out, the kernel stops, frees its tensor memory,
  *   records B200ATTN_ERR_TIMEOUT in a device status word and returns. The
  *   status word is read (and cleared) by b200attn_check.
- * - The library holds no device memory of its own beyond that status word.
+ * - The library holds no device memory of its own beyond that status word and
+ *   the fixed 256 KiB scratch array of b200attn_quantize_fp8_static.
  */
 #ifndef B200ATTN_H_
 #define B200ATTN_H_
@@ -146,6 +147,39 @@ int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale,
                           int B, int N, int H, int d,
                           int granularity, int hadamard,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * b200attn_quantize_fp8_static -- the per-head (B200ATTN_SCALE_PER_HEAD)
+ * quantizer of b200attn_quantize_fp8, for callers that cannot allocate device
+ * memory: code that runs inside a framework which owns the device heap (a
+ * caching allocator or a fixed memory budget) and may not call cudaMalloc on
+ * its own, or a latency-critical path where an allocation could synchronise
+ * the device or fail. This entry point allocates nothing: neither cudaMalloc,
+ * cudaFree nor any allocating library routine is called.
+ *
+ * There is no counterpart on the pages this library follows; it only moves
+ * the quantizer's scratch (one partial absmax per 128-token block of each
+ * (b, h)) into a static device array of 65536 floats (256 KiB), which every GPU
+ * that loads the library holds until the process exits.
+ *
+ * Arguments and results are those of b200attn_quantize_fp8 with
+ * granularity = B200ATTN_SCALE_PER_HEAD: codes and scales are bit-identical.
+ *
+ * - Capacity: B * H * ceil(N/128) must not exceed 65536; larger problems are
+ *   rejected with B200ATTN_ERR_WORKSPACE before anything is launched.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ * - Every call on a device shares the one array, which keeps the last call's
+ *   partial absmax values (each call overwrites the slots it reads, so nothing
+ *   needs clearing). Calls that overlap on the GPU (on different streams, or
+ *   from different threads) race on it and must be serialised by the caller.
+ *
+ * Errors: INVALID, UNSUPPORTED (d not 128/192), WORKSPACE (too large), CUDA.
+ */
+int b200attn_quantize_fp8_static(const void* x, void* x_fp8, float* scale,
+                                 int B, int N, int H, int d,
+                                 int hadamard, void* stream);
 
 /*
  * b200attn_check -- synchronise `stream`, then return and clear the device
