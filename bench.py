@@ -302,10 +302,11 @@ def time_path(path: Path, steps: int, warmup: int, settle_s: float, flush, dist_
     return step_ms, attn_ms
 
 
-def max_over_ranks(x: float, dist_on: bool) -> float:
+def max_over_ranks(x: float, dist_on: bool, device: str = "cuda") -> float:
+    """The slowest rank's value: every rank contributes its own timing, all get the max."""
     if not dist_on:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 

@@ -12,5 +12,6 @@ from ._binding import (  # noqa: F401
     load_library,
     quantize_fp8,
     quantize_workspace_bytes,
+    selftest_wait_timeout,
     version,
 )

@@ -55,6 +55,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.b200attn_strerror.argtypes = [i]
     lib.b200attn_version.restype = i
     lib.b200attn_version.argtypes = []
+    lib.b200attn_selftest_wait_timeout.restype = i
+    lib.b200attn_selftest_wait_timeout.argtypes = [i, vp]
     _lib = lib
     return lib
 
@@ -179,6 +181,13 @@ def attn_func(q, k, v, softmax_scale: float | None = None, causal: bool = True, 
 def check(stream=None) -> int:
     """Synchronise the stream and return/clear the library's device status word (0 = ok)."""
     return int(load_library().b200attn_check(_stream_handle(stream)))
+
+
+def selftest_wait_timeout(limit_us: int = 20000, stream=None) -> None:
+    """Launch the failure-path self-test kernel (a bounded wait that must run out)."""
+    rc = load_library().b200attn_selftest_wait_timeout(int(limit_us), _stream_handle(stream))
+    if rc != 0:
+        raise B200AttnError(rc, "b200attn_selftest_wait_timeout")
 
 
 def version() -> int:

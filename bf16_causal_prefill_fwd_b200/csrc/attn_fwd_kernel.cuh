@@ -149,14 +149,15 @@ __device__ __forceinline__ int unit_for(int k, int cta, int grid) {
 
 // Bounded mbarrier wait. Returns false if it gave up (2 s) or another role
 // already gave up; the first to give up records the timeout status.
-__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicCAS(&g_b200attn_status, 0, kStatusTimeout);
       return false;
@@ -422,11 +423,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int q_tile = 2 * x.pair + t;
       const int qrow = q_tile * kBM + r;
 
+      // FP8 scales. Per head: one multiplier on S and one on O. Per 128-token
+      // block: S of block i takes sq[q tile] * sk[i]; V's block scale sv[i] is
+      // folded into P as sv[i] / s_ref <= 1, where s_ref is the largest sv seen so
+      // far in this unit and O is kept in units of s_ref (rescaled when it grows).
       float c_log2 = p.scale_log2;
       float v_mult = 1.0f;
+      const float* ks_blk = nullptr;
+      const float* vs_blk = nullptr;
       if constexpr (FP8) {
-        c_log2 *= __ldg(p.q_scale + x.b * p.Hq + x.hq) * __ldg(p.k_scale + x.b * p.Hkv + x.hkv);
-        v_mult = __ldg(p.v_scale + x.b * p.Hkv + x.hkv);
+        if (p.per_block) {
+          const size_t kv_row = static_cast<size_t>(x.b * p.Hkv + x.hkv) * p.n_kv;
+          c_log2 *= __ldg(p.q_scale + static_cast<size_t>(x.b * p.Hq + x.hq) * p.n_kv + q_tile);
+          ks_blk = p.k_scale + kv_row;
+          vs_blk = p.v_scale + kv_row;
+        } else {
+          c_log2 *= __ldg(p.q_scale + x.b * p.Hq + x.hq) * __ldg(p.k_scale + x.b * p.Hkv + x.hkv);
+          v_mult = __ldg(p.v_scale + x.b * p.Hkv + x.hkv);
+        }
       }
       float m_run = -INFINITY, l_run = 0.0f;
 
@@ -474,14 +488,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mx0 = max3f(mx0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
         mx1 = max3f(mx1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
         const float mx = max3f(mx0, mx1, fmaxf(mx2, mx3));
-        const float m_new = fmaxf(m_run, mx * c_log2);
-        const bool need = m_new > m_run + C::T_LAG;
+        float c_blk = c_log2;  // S multiplier of this block (log2 units)
+        float lr = 0.0f;       // log2(sv[i] / s_ref), folded into P (per-block V scales)
+        float v_alpha = 1.0f;  // O rescale when s_ref grows
+        if constexpr (FP8) {
+          if (p.per_block) {
+            c_blk = c_log2 * __ldg(ks_blk + i);
+            const float sv = __ldg(vs_blk + i);
+            if (i == 0 || sv > v_mult) {
+              if (i > 0) v_alpha = v_mult / sv;
+              v_mult = sv;
+            }
+            lr = log2f(sv / v_mult);
+          }
+        }
+        const float m_new = fmaxf(m_run, mx * c_blk);
+        const bool need_m = m_new > m_run + C::T_LAG;
         float alpha = 1.0f;
-        if (need) {
+        if (need_m) {
           alpha = ex2_approx(m_run - m_new);
           m_run = m_new;
         }
         l_run *= alpha;
+        const bool need = need_m || v_alpha != 1.0f;
+        alpha *= v_alpha;
 
         // probabilities, packed in place (entry c/2 or c/4 is already consumed)
         float l_blk;
@@ -502,9 +532,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // acc: f16x2 partial sums of decode(code)/256 (8 adds per accumulator per block)
           uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
           if constexpr (LEANP) {
-            // w = clamp((8 (c*S - m_run + E) + 56) / 126, 0, 1); code = round(126 w)
-            const float A = c_log2 * (8.0f / 126.0f);
-            const float Bc = (8.0f * (C::E_SHIFT - m_run) + 56.0f) * (1.0f / 126.0f);
+            // w = clamp((8 (c*S - m_run + E + lr) + 56) / 126, 0, 1); code = round(126 w)
+            const float A = c_blk * (8.0f / 126.0f);
+            const float Bc = (8.0f * (C::E_SHIFT - m_run + lr) + 56.0f) * (1.0f / 126.0f);
 #pragma unroll
             for (int c = 0; c < 128; c += 4) {
               const float w0 = fma_sat(__uint_as_float(sr[c]), A, Bc);
@@ -521,13 +551,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               sr[c >> 2] = prmt(u01, u23, 0x6420u);  // bytes: code0, code1, code2, code3
             }
           } else {
-            const float nm = C::E_SHIFT - m_run;
+            const float nm = C::E_SHIFT - m_run + lr;
 #pragma unroll
             for (int c = 0; c < 128; c += 4) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, nm));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), c_log2, nm));
-              const float p2 = ex2_approx(fmaf(__uint_as_float(sr[c + 2]), c_log2, nm));
-              const float p3 = ex2_approx(fmaf(__uint_as_float(sr[c + 3]), c_log2, nm));
+              const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), c_blk, nm));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), c_blk, nm));
+              const float p2 = ex2_approx(fmaf(__uint_as_float(sr[c + 2]), c_blk, nm));
+              const float p3 = ex2_approx(fmaf(__uint_as_float(sr[c + 3]), c_blk, nm));
               const uint32_t w = static_cast<uint32_t>(pack_e4m3x2(p0, p1)) |
                                  (static_cast<uint32_t>(pack_e4m3x2(p2, p3)) << 16);
               const int jj = (c >> 1) & 7;
@@ -542,6 +572,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float s45 = f16x2_sum_f32(acc[4]) + f16x2_sum_f32(acc[5]);
           const float s67 = f16x2_sum_f32(acc[6]) + f16x2_sum_f32(acc[7]);
           l_blk = ((s01 + s23) + (s45 + s67)) * 256.0f;
+          if (lr != 0.0f) l_blk *= ex2_approx(-lr);  // back to unscaled probabilities
         }
         l_run += l_blk;
 
@@ -602,6 +633,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Failure-path self-test: one thread waits, through the same bounded wait as
+// the attention kernel, on an mbarrier that nothing ever arrives on. After
+// limit_ns it gives up, records B200ATTN_ERR_TIMEOUT in the status word and
+// returns; nothing traps and the context stays usable.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_addr(&bar), 1);
+    fence_mbar_init();
+    mbar_wait_slow(smem_addr(&bar), 0, &abort_flag, limit_ns);
   }
 }
 

@@ -127,7 +127,8 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
   const bool fp8 = dtype == B200ATTN_FP8_E4M3;
   if (fp8) {
     if (!q_scale || !k_scale || !v_scale) return B200ATTN_ERR_INVALID;
-    if (scale_granularity != B200ATTN_SCALE_PER_HEAD) return B200ATTN_ERR_UNSUPPORTED;
+    if (scale_granularity != B200ATTN_SCALE_PER_HEAD && scale_granularity != B200ATTN_SCALE_PER_BLOCK)
+      return B200ATTN_ERR_UNSUPPORTED;
   }
   // index arithmetic inside the kernels is 32-bit over (b, n, h) rows
   if (static_cast<int64_t>(B) * N * (Hq > Hkv ? Hq : Hkv) >= (int64_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
@@ -253,6 +254,16 @@ int b200attn_quantize_fp8_static(const void* x, void* x_fp8, float* scale, int B
                     : launch_quant<128, false>(x, x_fp8, scale, B, N, H, B200ATTN_SCALE_PER_HEAD, scratch, st);
   return hadamard ? launch_quant<192, true>(x, x_fp8, scale, B, N, H, B200ATTN_SCALE_PER_HEAD, scratch, st)
                   : launch_quant<192, false>(x, x_fp8, scale, B, N, H, B200ATTN_SCALE_PER_HEAD, scratch, st);
+}
+
+int b200attn_selftest_wait_timeout(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 10000000) return B200ATTN_ERR_INVALID;
+  int sm_count = 0;
+  const int dev_rc = device_ok(&sm_count);
+  if (dev_rc != B200ATTN_OK) return dev_rc;
+  b200::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
 }
 
 int b200attn_check(void* stream) {

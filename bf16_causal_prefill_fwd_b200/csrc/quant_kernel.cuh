@@ -8,11 +8,13 @@
 // 开源 ZYFA …", "ZYFA 的 FP8 注意力有多准确？" (a Hadamard rotation of Q and K
 // roughly halves the input-quantisation error at ~0.1% attention time).
 //
-// HBM-bound: one warp per 128- or 192-element row, 16 rows per warp, 8 warps
-// per CTA, one CTA per (b, h, 128-token block). A row is read with 8-byte
-// (d=128 part) and 4-byte (d=192 tail) loads, so a warp touches a contiguous
-// 256/384-byte row. The rotated values stay in registers between the absmax
-// reduction and the encode, so x is read once per pass.
+// HBM-bound: one CTA of 8 warps per (b, h, 128-token block). A row is held by
+// 16 lanes: for d = 128 each lane loads 8 bf16 (16 bytes), so one warp
+// instruction moves two rows; for d = 192 lanes 0-15 load 8 of the first 128
+// and lanes 16-31 load 4 of the 64-wide tail. Every load of the block is
+// issued before any arithmetic (row indices are clamped, never branched on),
+// which keeps 32 KiB per CTA in flight. The rotated values stay in registers
+// between the absmax reduction and the encode, so x is read once per pass.
 //
 // Arithmetic contract (identical on every call, so codes are reproducible):
 //   rotation: radix-2 butterflies of widths 1, 2, 4, ... (the lower element of
@@ -29,77 +31,101 @@
 namespace b200 {
 
 constexpr int kQuantThreads = 256;
-constexpr int kQuantRowsPerWarp = 16;
 constexpr int kQuantBlock = 128;  // tokens per scale block
 
-// One row (d = 128 or 192) held by a warp: a[e] = element 4*lane+e of the first
-// 128, t[e] = element 128+2*lane+e of the 64-wide tail (d = 192 only).
+// Rows of one block held by a warp: d = 128 -> 8 row pairs (lanes 0-15: even
+// row of the pair, 16-31: odd row); d = 192 -> 16 rows, one per instruction.
 template <int D>
-struct RowRegs {
-  float a[4];
-  float t[2];
+struct QuantLayout {
+  static constexpr int ROWS_PER_INSTR = D == 128 ? 2 : 1;
+  static constexpr int ITERS = kQuantBlock / 8 / ROWS_PER_INSTR;  // per warp: 16 rows
 };
 
-template <int D, bool HAD>
-__device__ __forceinline__ void load_row(const __nv_bfloat16* row, int lane, RowRegs<D>& v) {
-  const uint2 raw = *reinterpret_cast<const uint2*>(row + 4 * lane);
-  const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-  const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-  v.a[0] = __low2float(p0);
-  v.a[1] = __high2float(p0);
-  v.a[2] = __low2float(p1);
-  v.a[3] = __high2float(p1);
-  if constexpr (D == 192) {
-    const uint32_t rt = *reinterpret_cast<const uint32_t*>(row + 128 + 2 * lane);
-    const __nv_bfloat162 pt = *reinterpret_cast<const __nv_bfloat162*>(&rt);
-    v.t[0] = __low2float(pt);
-    v.t[1] = __high2float(pt);
+__device__ __forceinline__ void bf16x8_to_float(const uint4& raw, float (&v)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
-  if constexpr (HAD) {
-    // width 1 and 2: inside the thread
-    float b0 = __fadd_rn(v.a[0], v.a[1]), b1 = __fsub_rn(v.a[0], v.a[1]);
-    float b2 = __fadd_rn(v.a[2], v.a[3]), b3 = __fsub_rn(v.a[2], v.a[3]);
-    v.a[0] = __fadd_rn(b0, b2);
-    v.a[2] = __fsub_rn(b0, b2);
-    v.a[1] = __fadd_rn(b1, b3);
-    v.a[3] = __fsub_rn(b1, b3);
-    // widths 4 .. 64: partner lane differs in bit (width / 4)
-#pragma unroll
-    for (int m = 1; m <= 16; m <<= 1) {
-      const bool upper = (lane & m) != 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float o = __shfl_xor_sync(0xffffffffu, v.a[e], m);
-        v.a[e] = upper ? __fsub_rn(o, v.a[e]) : __fadd_rn(v.a[e], o);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) v.a[e] = __fmul_rn(v.a[e], 0.08838834764831845f);
-    if constexpr (D == 192) {
-      float c0 = __fadd_rn(v.t[0], v.t[1]), c1 = __fsub_rn(v.t[0], v.t[1]);
-      v.t[0] = c0;
-      v.t[1] = c1;
-      // widths 2 .. 32: partner lane differs in bit (width / 2)
-#pragma unroll
-      for (int m = 1; m <= 16; m <<= 1) {
-        const bool upper = (lane & m) != 0;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float o = __shfl_xor_sync(0xffffffffu, v.t[e], m);
-          v.t[e] = upper ? __fsub_rn(o, v.t[e]) : __fadd_rn(v.t[e], o);
-        }
-      }
-      v.t[0] = __fmul_rn(v.t[0], 0.125f);
-      v.t[1] = __fmul_rn(v.t[1], 0.125f);
+}
+
+// Load the 8 (or 4) elements this lane holds of one row; `row` is clamped by the caller.
+template <int D>
+__device__ __forceinline__ void load_lane(const __nv_bfloat16* row, int lane, float (&v)[8]) {
+  if constexpr (D == 128) {
+    bf16x8_to_float(*reinterpret_cast<const uint4*>(row + 8 * (lane & 15)), v);
+  } else {
+    if (lane < 16) {
+      bf16x8_to_float(*reinterpret_cast<const uint4*>(row + 8 * lane), v);
+    } else {
+      const uint2 raw = *reinterpret_cast<const uint2*>(row + 128 + 4 * (lane - 16));
+      v[0] = __uint_as_float(raw.x << 16);
+      v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+      v[2] = __uint_as_float(raw.y << 16);
+      v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+      v[4] = v[5] = v[6] = v[7] = 0.0f;
     }
   }
 }
 
+// In-place normalised Walsh-Hadamard transform of this lane's segment. Lanes
+// 0-15 (and, for d = 128, lanes 16-31) hold 8 consecutive elements of a
+// 128-wide row; for d = 192 lanes 16-31 hold 4 consecutive elements of the
+// 64-wide tail. Every element ends up as the same sequence of fp32 additions
+// and subtractions as the textbook in-place algorithm.
 template <int D>
-__device__ __forceinline__ float row_absmax(const RowRegs<D>& v) {
-  float m = fmaxf(fmaxf(fabsf(v.a[0]), fabsf(v.a[1])), fmaxf(fabsf(v.a[2]), fabsf(v.a[3])));
-  if constexpr (D == 192) m = fmaxf(m, fmaxf(fabsf(v.t[0]), fabsf(v.t[1])));
-  return m;
+__device__ __forceinline__ void rotate_lane(int lane, float (&v)[8]) {
+  const bool tail = (D == 192) && lane >= 16;
+  // widths 1, 2 (and 4 for 8-element segments) inside the thread
+#pragma unroll
+  for (int h = 1; h <= 4; h <<= 1) {
+    if (h == 4 && tail) break;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if ((e & h) == 0) {
+        const float a = v[e], b = v[e + h];
+        v[e] = __fadd_rn(a, b);
+        v[e + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+  // remaining widths across lanes: partner lane differs in bit m of the lane index
+#pragma unroll
+  for (int m = 1; m <= 8; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
+      v[e] = upper ? __fsub_rn(o, v[e]) : __fadd_rn(v[e], o);
+    }
+  }
+  const float c = tail ? 0.125f : 0.08838834764831845f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], c);
+}
+
+template <int D, bool HAD>
+__device__ __forceinline__ void load_block(const __nv_bfloat16* __restrict__ x, int b, int h, int blk, int N, int H,
+                                           int warp, int lane, float (&v)[QuantLayout<D>::ITERS][8], float& amax) {
+  using L = QuantLayout<D>;
+  const int sub = (D == 128) ? (lane >> 4) : 0;
+#pragma unroll
+  for (int it = 0; it < L::ITERS; ++it) {
+    const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
+    const int rc = row < N ? row : N - 1;
+    load_lane<D>(x + (static_cast<size_t>(b) * N + rc) * H * D + static_cast<size_t>(h) * D, lane, v[it]);
+  }
+  amax = 0.0f;
+#pragma unroll
+  for (int it = 0; it < L::ITERS; ++it) {
+    if constexpr (HAD) rotate_lane<D>(lane, v[it]);
+    const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
+    if (row < N) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[it][e]));
+    }
+  }
 }
 
 __device__ __forceinline__ float block_max(float m, float* red) {
@@ -122,19 +148,11 @@ __global__ void __launch_bounds__(kQuantThreads)
   __shared__ float red[kQuantThreads / 32];
   const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nblk = gridDim.x;
-  float m = 0.0f;
-#pragma unroll 4
-  for (int j = 0; j < kQuantRowsPerWarp; ++j) {
-    const int row = blk * kQuantBlock + warp * kQuantRowsPerWarp + j;
-    if (row < N) {  // warp-uniform
-      RowRegs<D> v;
-      load_row<D, HAD>(x + (static_cast<size_t>(b) * N + row) * H * D + static_cast<size_t>(h) * D, lane, v);
-      m = fmaxf(m, row_absmax<D>(v));
-    }
-  }
+  float v[QuantLayout<D>::ITERS][8];
+  float m;
+  load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, v, m);
   m = block_max(m, red);
-  if (threadIdx.x == 0) partial[(static_cast<size_t>(b) * H + h) * nblk + blk] = m;
+  if (threadIdx.x == 0) partial[(static_cast<size_t>(b) * H + h) * gridDim.x + blk] = m;
 }
 
 // Encode one 128-token block. PER_HEAD: amax is the max of the partials of
@@ -143,21 +161,15 @@ template <int D, bool HAD, bool PER_HEAD>
 __global__ void __launch_bounds__(kQuantThreads)
     quant_encode_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
                         float* __restrict__ scale, const float* __restrict__ partial, int N, int H) {
+  using L = QuantLayout<D>;
   __shared__ float red[kQuantThreads / 32];
   const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nblk = gridDim.x;
 
-  RowRegs<D> v[kQuantRowsPerWarp];
-  float m = 0.0f;
-#pragma unroll
-  for (int j = 0; j < kQuantRowsPerWarp; ++j) {
-    const int row = blk * kQuantBlock + warp * kQuantRowsPerWarp + j;
-    if (row < N) {
-      load_row<D, HAD>(x + (static_cast<size_t>(b) * N + row) * H * D + static_cast<size_t>(h) * D, lane, v[j]);
-      m = fmaxf(m, row_absmax<D>(v[j]));
-    }
-  }
+  float v[L::ITERS][8];
+  float m;
+  load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, v, m);
   if constexpr (PER_HEAD) {
     m = 0.0f;
     const float* ph = partial + (static_cast<size_t>(b) * H + h) * nblk;
@@ -174,17 +186,20 @@ __global__ void __launch_bounds__(kQuantThreads)
       scale[(static_cast<size_t>(b) * H + h) * nblk + blk] = sc;
     }
   }
+  const int sub = (D == 128) ? (lane >> 4) : 0;
 #pragma unroll
-  for (int j = 0; j < kQuantRowsPerWarp; ++j) {
-    const int row = blk * kQuantBlock + warp * kQuantRowsPerWarp + j;
+  for (int it = 0; it < L::ITERS; ++it) {
+    const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
     if (row < N) {
       uint8_t* dst = y + (static_cast<size_t>(b) * N + row) * H * D + static_cast<size_t>(h) * D;
-      const uint32_t lo = pack_e4m3x2(__fmul_rn(v[j].a[0], inv), __fmul_rn(v[j].a[1], inv));
-      const uint32_t hi = pack_e4m3x2(__fmul_rn(v[j].a[2], inv), __fmul_rn(v[j].a[3], inv));
-      *reinterpret_cast<uint32_t*>(dst + 4 * lane) = lo | (hi << 16);
-      if constexpr (D == 192) {
-        *reinterpret_cast<uint16_t*>(dst + 128 + 2 * lane) =
-            pack_e4m3x2(__fmul_rn(v[j].t[0], inv), __fmul_rn(v[j].t[1], inv));
+      uint32_t c[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        c[q] = pack_e4m3x2(__fmul_rn(v[it][2 * q], inv), __fmul_rn(v[it][2 * q + 1], inv));
+      if (D == 128 || lane < 16) {
+        *reinterpret_cast<uint2*>(dst + 8 * (lane & 15)) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+      } else {
+        *reinterpret_cast<uint32_t*>(dst + 128 + 4 * (lane - 16)) = c[0] | (c[1] << 16);
       }
     }
   }

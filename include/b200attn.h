@@ -188,6 +188,17 @@ int b200attn_quantize_fp8_static(const void* x, void* x_fp8, float* scale,
  */
 int b200attn_check(void* stream);
 
+/*
+ * b200attn_selftest_wait_timeout -- exercise the failure path on purpose.
+ * Launches (on `stream`) a one-thread kernel that waits, with the same bounded
+ * wait the attention kernel uses, on a barrier nothing arrives on; after
+ * limit_us microseconds (1 .. 10^7) it gives up, records B200ATTN_ERR_TIMEOUT
+ * in the device status word and returns. It never traps, so the context stays
+ * usable: the next b200attn_check returns B200ATTN_ERR_TIMEOUT (and clears it),
+ * and later calls run normally. For tests of error handling.
+ */
+int b200attn_selftest_wait_timeout(int limit_us, void* stream);
+
 /* Static description of a status code; never NULL. */
 const char* b200attn_strerror(int code);
 

@@ -1,0 +1,51 @@
+"""The N>1 plumbing of bench.py on CPU with gloo (world size 2): every rank
+gets the slowest rank's time, and the reference arm runs on rank 0 only."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        results[rank] = bench.max_over_ranks(1.5 + rank, True, device="cpu")
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_with_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_worker, args=(r, world, port, results)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+            assert p.exitcode == 0
+        assert dict(results) == {0: 2.5, 1: 2.5}
+
+
+def test_reference_arm_other_ranks_do_no_work(capsys):
+    import bench
+
+    class A:
+        workload, n, warmup, steps = "tiny", None, 3, 1
+    bench.run_reference(A(), rank=1, world=2)
+    assert capsys.readouterr().out == ""

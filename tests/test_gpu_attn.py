@@ -109,6 +109,43 @@ def test_fp8_matches_oracle(shape, causal, fp8_p):
     check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
 
 
+PER_BLOCK_SHAPES = [(1, 4, 2, 300, 128), (2, 2, 1, 700, 128), (1, 4, 4, 520, 192)]
+
+
+@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
+@pytest.mark.parametrize("shape", PER_BLOCK_SHAPES)
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_per_block_scales_match_oracle(shape, causal, fp8_p):
+    """Scales per (b, h, 128-token block); V blocks get very different magnitudes so the
+    kernel's per-block V reference grows and O is rescaled."""
+    B, Hq, Hkv, N, dqk = shape
+    q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + 7))
+    gain = torch.tensor([0.05, 3.0, 0.5, 20.0, 1.0, 0.01])[(torch.arange(N) // 128) % 6]
+    v = (v.float() * gain[None, :, None, None]).to(torch.bfloat16)
+    k = (k.float() * gain.flip(0)[None, :, None, None].sqrt()).to(torch.bfloat16)
+    codes, deq = oracle_fp8_inputs(q, k, v, granularity="block")
+    q8, sq, k8, sk, v8, sv = to_gpu_fp8(codes)
+    o, lse = b2.attn_fwd(q8, k8, v8, q_scale=sq, k_scale=sk, v_scale=sv, causal=causal,
+                         scale_granularity="block", return_lse=True)
+    assert b2.check() == 0
+    ref, ref_lse = oracle.attention(*deq, causal=causal)
+    err = oracle.rel_rms(f32(o), ref)
+    assert err <= FP8_TOL, err
+    check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
+
+
+def test_fp8_per_block_equals_per_head_when_scales_agree():
+    """Per-block scales that all equal the per-head scale give bitwise the same output."""
+    q, k, v = workloads.draw(workloads.gaussian(1, 4, 2, 384, 128, 128, seed=9))
+    codes, _ = oracle_fp8_inputs(q, k, v, granularity="head")
+    q8, sq, k8, sk, v8, sv = to_gpu_fp8(codes)
+    o_head = b2.attn_fwd(q8, k8, v8, q_scale=sq, k_scale=sk, v_scale=sv)
+    rep = lambda s: s[:, :, None].expand(-1, -1, 3).contiguous()
+    o_blk = b2.attn_fwd(q8, k8, v8, q_scale=rep(sq), k_scale=rep(sk), v_scale=rep(sv), scale_granularity="block")
+    assert b2.check() == 0
+    assert torch.equal(o_head, o_blk)
+
+
 @pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
 def test_tiny_workload_both_dtypes(fp8_p):
     w = workloads.tiny()
