@@ -333,7 +333,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         value = world * w.flops / (ms * 1e-3) / 1e12
         achieved = w.flops / (ams * 1e-3) / 1e12
         peak = bf16_peak * (2.0 if dtype == "fp8" else 1.0)
-        kernel_key = f"attn_fwd_kernel<{w.d_qk},{w.d_v},{'fp8' if dtype == 'fp8' else 'bf16'}>"
+        fp8_p = os.environ.get("B200ATTN_FP8_P", "lean")
+        kernel_key = (f"attn_fwd_kernel<{w.d_qk},{w.d_v},fp8,{'mufu' if fp8_p == 'mufu' else 'lean'}>"
+                      if dtype == "fp8" else f"attn_fwd_kernel<{w.d_qk},{w.d_v},bf16>")
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic_for(kernel_key, w.name),
                 "kernel": kernel_key, "kernel_ms": ams,
