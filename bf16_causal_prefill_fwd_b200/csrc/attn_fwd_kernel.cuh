@@ -16,24 +16,34 @@
 // fixed key order: results are bitwise reproducible.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles, then K_0, V_0, K_1, V_1, ... into a ring
-//   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
-//   warps 2-3   idle
+//   warp 0      TMA producer of Q tiles and of the K ring
+//   warps 1, 2  MMA issuers (one thread each; warp 2 only with P in shared
+//               memory), see below
+//   warp 3      TMA producer of the V ring
 //   warps 4-7   softmax + epilogue for tile 0 (one thread per query row)
 //   warps 8-11  softmax + epilogue for tile 1
-// The two softmax warpgroups alternate the way the pages' two-wave ping-pong
-// does ("ZYFA 如何工作？", 双波乒乓调度): while one computes probabilities for
-// block i the tensor core runs the other tile's PV and next QK^T. On sm_100 the
-// MMA completion is tracked in hardware (tcgen05.commit -> mbarrier), so the
-// overlap needs no instruction-order scheduling.
+// With P in shared memory two MMA issuers split by role (warp 1 all QK^T, warp
+// 2 all PV): they wait on different events (scores consumed, probabilities
+// ready), so neither holds up the other's MMAs, and the tensor core runs what
+// both have queued. With P in TMEM, warp 1 alone issues both tiles' MMAs,
+// each tile's PV followed by its next QK^T.
+// The two softmax warpgroups work side by side the way the pages' two-wave
+// ping-pong does ("ZYFA 如何工作？", 双波乒乓调度): while one computes
+// probabilities the tensor core runs the other tile's matrix products. On
+// sm_100 MMA completion is tracked in hardware (tcgen05.commit -> mbarrier),
+// so the overlap needs no instruction-order scheduling.
 //
-// Tensor memory (512 columns x 128 lanes, fp32):
-//   [  0,128) S_0, with P_0 written over its first columns
-//   [128,256) S_1 / P_1
-//   [256,384) O_0 accumulator (d_v = 128)
-//   [384,512) O_1 accumulator
-// MMAs issued by one thread execute in order, so P_t (read by PV_t,i) is never
-// overwritten by S_t,i+1 before that PV has consumed it.
+// Tensor memory (512 columns x 128 lanes, fp32): [0,128) S_0, [128,256) S_1,
+// [256,384) O_0, [384,512) O_1.
+//
+// Where the probabilities P go (template switch PS):
+//  * PS (FP8): P is written to shared memory in the 128-byte-swizzled K-major
+//    layout the tensor core reads, and PV takes both operands from shared
+//    memory. The softmax frees S_t as soon as it has copied the scores into
+//    registers, so S_t for the next key block is computed while the
+//    probabilities of this block are still being formed.
+//  * otherwise (BF16): P is written over the first columns of S_t in TMEM and
+//    PV reads it from there; S_t for the next block starts once PV_t has read P.
 //
 // Online softmax per row (log2 domain, c = s * log2(e) [* q/k scales]):
 //   m_blk = max_j S_ij; m_new = max(m_run, c * m_blk)
@@ -48,10 +58,11 @@
 //  * MUFU: P = e4m3(ex2(x)), round to nearest even.
 //  * Lean P ("ZYFA 如何工作？", Lean P：用一次乘加代替指数运算): read as an
 //    integer, the e4m3 code of 2^x is close to 8x + 56 (+8 per doubling), so the
-//    code is built with fused multiply-adds and no exponential: one saturating
-//    FFMA gives w = clamp((8x + 56)/126, 0, 1), a pack to f16x2 and one f16x2
-//    FMA with the magic 1536 (f16 spacing 1 in [1024, 2048)) leave
-//    round(126 w) in the low byte of each lane, and one PRMT gathers four codes.
+//    code is built with fused multiply-adds and no exponential: one packed FFMA
+//    gives w = (8x + 56)/126 for two scores, a convert to f16x2 clamps negative
+//    w to 0 (w <= 120/126 by the choice of T and E), and one f16x2 FMA with the
+//    magic 1536 (f16 spacing 1 in [1024, 2048)) leaves round(126 w) in the low
+//    byte of each lane; one PRMT gathers four codes.
 // Either way l is the sum of the rounded probabilities the PV MMA multiplies
 // ("逐块缩放与舍入行和": divide by the sum of the rounded probabilities): the
 // bits (code << 7) read as an f16 are exactly decode(code) / 256 for every
@@ -89,23 +100,35 @@ struct AttnParams {
   float* lse;
 };
 
-template <int DQK, int DV, bool FP8, bool LEANP = false>
+template <int DQK, int DV, bool FP8, bool LEANP = false, bool P_SMEM = true>
 struct AttnCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int CHUNK_ELEMS = 128 / ESZ;  // elements in one 128-byte swizzled row
   static constexpr int CHUNK_BYTES = kBM * 128;  // one 128-row x 128-byte swizzle column: 16 KiB
   static constexpr int QK_CHUNKS = (DQK + CHUNK_ELEMS - 1) / CHUNK_ELEMS;
   static constexpr int V_CHUNKS = (DV + CHUNK_ELEMS - 1) / CHUNK_ELEMS;
+  static constexpr int P_CHUNKS = kBN / CHUNK_ELEMS;  // P tile [128 rows, 128 keys]
   static constexpr int Q_BYTES = QK_CHUNKS * CHUNK_BYTES;
   static constexpr int K_BYTES = QK_CHUNKS * CHUNK_BYTES;
   static constexpr int V_BYTES = V_CHUNKS * CHUNK_BYTES;
+  static constexpr int P_BYTES = P_CHUNKS * CHUNK_BYTES;
   static constexpr int STAGE_BYTES = K_BYTES > V_BYTES ? K_BYTES : V_BYTES;
   static constexpr int MMA_K = FP8 ? 32 : 16;  // reduction depth of one tcgen05.mma
-  static constexpr int STAGES_FIT = (200 * 1024 - 2 * Q_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int NUM_BARS = 2 + 2 + 2 * STAGES + 2 + 2 + 2 + 2 + 1;
-  static constexpr int SMEM_BYTES = 2 * Q_BYTES + STAGES * STAGE_BYTES + 1024 /*bars*/ + 1024 /*align*/;
-  // P columns: bf16 packs 2 keys per 32-bit column, e4m3 packs 4.
+  // P in shared memory (see the file comment); P buffers per tile.
+  static constexpr bool PS = P_SMEM && FP8;
+  static constexpr int PB = PS ? (DQK == 128 ? 2 : 1) : 0;
+  static constexpr int PBX = PS ? PB : 1;  // P-full / P-done barriers per tile
+  // Separate K and V rings, sized from what shared memory has left.
+  static constexpr int SMEM_AVAIL = 227 * 1024 - 2048;  // minus barriers and alignment slack
+  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BYTES - 2 * PB * P_BYTES;
+  static constexpr int RING_PAIRS = RING_AVAIL / (K_BYTES + V_BYTES);
+  static constexpr int SV = RING_PAIRS >= 2 ? (RING_PAIRS > 4 ? 4 : RING_PAIRS) : 1;
+  static constexpr int SK_FIT = (RING_AVAIL - SV * V_BYTES) / K_BYTES;
+  static constexpr int SK = SK_FIT > 6 ? 6 : SK_FIT;
+  static constexpr int NUM_BARS = 2 + 2 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
+  static constexpr int SMEM_BYTES = 2 * Q_BYTES + 2 * PB * P_BYTES + SK * K_BYTES + SV * V_BYTES +
+                                    1024 /*bars*/ + 1024 /*align*/;
+  // P columns in TMEM (non-PS): bf16 packs 2 keys per 32-bit column, e4m3 packs 4.
   static constexpr int P_COLS = kBN * ESZ / 4;
   static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
   static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
@@ -113,7 +136,8 @@ struct AttnCfg {
   static constexpr uint32_t IDESC_QK = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, kBN, false);
   static constexpr uint32_t IDESC_PV = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DV, true);
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
-  static_assert(STAGES >= 2, "need at least two K/V stages");
+  static_assert(SK >= 2 && SV >= 1, "K/V rings");
+  static_assert(8 * NUM_BARS + 8 <= 1024, "barrier area");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -170,11 +194,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort_flag);
 }
 
-template <int DQK, int DV, bool FP8, bool LEANP>
+template <int DQK, int DV, bool FP8, bool LEANP, bool P_SMEM>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<DQK, DV, FP8, LEANP>;
+  using C = AttnCfg<DQK, DV, FP8, LEANP, P_SMEM>;
   extern __shared__ uint8_t smem_raw[];
 
   // 1024-byte aligned base (128-byte swizzle atoms repeat every 1024 bytes).
@@ -182,23 +206,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
 
-  const uint32_t sQ = base_u32;                         // 2 query tiles
-  const uint32_t sRing = base_u32 + 2 * C::Q_BYTES;     // K/V ring
-  const uint32_t sBar = sRing + C::STAGES * C::STAGE_BYTES;
+  const uint32_t sQ = base_u32;                              // 2 query tiles
+  const uint32_t sP = sQ + 2 * C::Q_BYTES;                   // [tile][PB] probability tiles (PS)
+  const uint32_t sK = sP + 2 * C::PB * C::P_BYTES;           // K ring
+  const uint32_t sV = sK + C::SK * C::K_BYTES;               // V ring
+  const uint32_t sBar = sV + C::SV * C::V_BYTES;
   uint8_t* bar_ptr = base + (sBar - base_u32);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NUM_BARS + 4);
 
   // barrier addresses
-  const uint32_t bQFull = sBar;                          // [2]  TMA -> MMA
-  const uint32_t bQEmpty = bQFull + 16;                  // [2]  MMA -> TMA
-  const uint32_t bKVFull = bQEmpty + 16;                 // [S]  TMA -> MMA
-  const uint32_t bKVEmpty = bKVFull + 8 * C::STAGES;     // [S]  MMA -> TMA
-  const uint32_t bSFull = bKVEmpty + 8 * C::STAGES;      // [2]  MMA -> softmax
-  const uint32_t bPFull = bSFull + 16;                   // [2]  softmax -> MMA (128 arrivals)
-  const uint32_t bOFull = bPFull + 16;                   // [2]  MMA -> epilogue
-  const uint32_t bOEmpty = bOFull + 16;                  // [2]  epilogue -> MMA (128 arrivals)
-  const uint32_t bDrain = bOEmpty + 16;                  // [1]  MMA drain at exit
+  const uint32_t bQFull = sBar;                          // [2]  TMA -> QK issuer
+  const uint32_t bQEmpty = bQFull + 16;                  // [2]  QK issuer -> TMA
+  const uint32_t bKFull = bQEmpty + 16;                  // [SK] TMA -> QK issuer
+  const uint32_t bKEmpty = bKFull + 8 * C::SK;           // [SK] QK issuer -> TMA
+  const uint32_t bVFull = bKEmpty + 8 * C::SK;           // [SV] TMA -> PV issuer
+  const uint32_t bVEmpty = bVFull + 8 * C::SV;           // [SV] PV issuer -> TMA
+  const uint32_t bSFull = bVEmpty + 8 * C::SV;           // [2]  QK issuer -> softmax
+  const uint32_t bSFree = bSFull + 16;                   // [2]  softmax -> QK issuer (128 arrivals; PS)
+  // P full (softmax -> PV issuer, 128 arrivals) and P done (PV issuer -> softmax
+  // and, without PS, -> QK issuer), per tile and P buffer. One barrier per
+  // buffer keeps a softmax that runs a block ahead from completing two phases of
+  // the barrier the PV issuer is about to wait on.
+  const uint32_t bPFull = bSFree + 16;                   // [2][PBX]
+  const uint32_t bPDone = bPFull + 16 * C::PBX;          // [2][PBX]
+  const uint32_t bOFull = bPDone + 16 * C::PBX;          // [2]  PV issuer -> epilogue
+  const uint32_t bOEmpty = bOFull + 16;                  // [2]  epilogue -> PV issuer (128 arrivals)
+  const uint32_t bDrain = bOEmpty + 16;                  // [2]  issuers' drains at exit
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -209,15 +243,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(bQFull + 8 * t, 1);
         mbar_init(bQEmpty + 8 * t, 1);
         mbar_init(bSFull + 8 * t, 1);
-        mbar_init(bPFull + 8 * t, 128);
+        mbar_init(bSFree + 8 * t, 128);
+        for (int b = 0; b < C::PBX; ++b) {
+          mbar_init(bPFull + 8 * (t * C::PBX + b), 128);
+          mbar_init(bPDone + 8 * (t * C::PBX + b), 1);
+        }
         mbar_init(bOFull + 8 * t, 1);
         mbar_init(bOEmpty + 8 * t, 128);
+        mbar_init(bDrain + 8 * t, 1);
       }
-      for (int s = 0; s < C::STAGES; ++s) {
-        mbar_init(bKVFull + 8 * s, 1);
-        mbar_init(bKVEmpty + 8 * s, 1);
+      for (int s = 0; s < C::SK; ++s) {
+        mbar_init(bKFull + 8 * s, 1);
+        mbar_init(bKEmpty + 8 * s, 1);
       }
-      mbar_init(bDrain, 1);
+      for (int s = 0; s < C::SV; ++s) {
+        mbar_init(bVFull + 8 * s, 1);
+        mbar_init(bVEmpty + 8 * s, 1);
+      }
       *abort_flag = 0;
       fence_mbar_init();
       prefetch_tmap(&tmQ);
@@ -233,172 +275,218 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0: Q tiles and K blocks; warp 3: V blocks. Each walks the same unit
+    // sequence and fills its ring in the order the issuers use it.
     if (lane == 0) {
+      const bool is_k = warp == 0;
       const uint64_t pol_kv = policy_evict_last();
       const uint64_t pol_q = policy_evict_first();
-      uint32_t kv_it = 0;
+      const int nslot = is_k ? C::SK : C::SV;
+      const uint32_t ring = is_k ? sK : sV;
+      const uint32_t slot_bytes = is_k ? C::K_BYTES : C::V_BYTES;
+      const uint32_t bFull = is_k ? bKFull : bVFull, bEmpty = is_k ? bKEmpty : bVEmpty;
+      const CUtensorMap* tm = is_k ? &tmK : &tmV;
+      const int chunks = is_k ? C::QK_CHUNKS : C::V_CHUNKS;
+      uint32_t it = 0;
       uint32_t qe_par[2] = {0, 0};
       bool first = true, ok = true;
       for (int k = 0; ok; ++k) {
         const int u = unit_for(k, blockIdx.x, gridDim.x);
         if (u >= p.n_units) break;
         const Unit x = decode_unit(u, p);
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!first) {
-            ok = mbar_wait(bQEmpty + 8 * t, qe_par[t], abort_flag);
-            qe_par[t] ^= 1;
-            if (!ok) break;
-          }
-          const uint32_t bar = bQFull + 8 * t;
-          mbar_arrive_expect_tx(bar, C::Q_BYTES);
-#pragma unroll
-          for (int c = 0; c < C::QK_CHUNKS; ++c)
-            tma_load_4d_hint(sQ + t * C::Q_BYTES + c * C::CHUNK_BYTES, &tmQ, bar, c * C::CHUNK_ELEMS,
-                             x.hq, (2 * x.pair + t) * kBM, x.b, pol_q);
-        }
-        for (int i = 0; i < x.n1 && ok; ++i) {
-          for (int kv = 0; kv < 2; ++kv) {  // 0: K_i, 1: V_i
-            const uint32_t s = kv_it % C::STAGES;
-            if (kv_it >= static_cast<uint32_t>(C::STAGES)) {
-              ok = mbar_wait(bKVEmpty + 8 * s, ((kv_it / C::STAGES) - 1) & 1, abort_flag);
+        if (is_k) {
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!first) {
+              ok = mbar_wait(bQEmpty + 8 * t, qe_par[t], abort_flag);
+              qe_par[t] ^= 1;
               if (!ok) break;
             }
-            const uint32_t bar = bKVFull + 8 * s;
-            const uint32_t dst = sRing + s * C::STAGE_BYTES;
-            if (kv == 0) {
-              mbar_arrive_expect_tx(bar, C::K_BYTES);
+            const uint32_t bar = bQFull + 8 * t;
+            mbar_arrive_expect_tx(bar, C::Q_BYTES);
 #pragma unroll
-              for (int c = 0; c < C::QK_CHUNKS; ++c)
-                tma_load_4d_hint(dst + c * C::CHUNK_BYTES, &tmK, bar, c * C::CHUNK_ELEMS, x.hkv,
-                                 i * kBN, x.b, pol_kv);
-            } else {
-              mbar_arrive_expect_tx(bar, C::V_BYTES);
-#pragma unroll
-              for (int c = 0; c < C::V_CHUNKS; ++c)
-                tma_load_4d_hint(dst + c * C::CHUNK_BYTES, &tmV, bar, c * C::CHUNK_ELEMS, x.hkv,
-                                 i * kBN, x.b, pol_kv);
-            }
-            ++kv_it;
+            for (int c = 0; c < C::QK_CHUNKS; ++c)
+              tma_load_4d_hint(sQ + t * C::Q_BYTES + c * C::CHUNK_BYTES, &tmQ, bar, c * C::CHUNK_ELEMS, x.hq,
+                               (2 * x.pair + t) * kBM, x.b, pol_q);
           }
+        }
+        for (int j = 0; j < x.n1 && ok; ++j, ++it) {
+          const uint32_t s = it % nslot;
+          if (it >= static_cast<uint32_t>(nslot) && !(ok = mbar_wait(bEmpty + 8 * s, ((it / nslot) - 1) & 1, abort_flag)))
+            break;
+          const uint32_t bar = bFull + 8 * s;
+          mbar_arrive_expect_tx(bar, slot_bytes);
+          for (int c = 0; c < chunks; ++c)
+            tma_load_4d_hint(ring + s * slot_bytes + c * C::CHUNK_BYTES, tm, bar, c * C::CHUNK_ELEMS, x.hkv, j * kBN,
+                             x.b, pol_kv);
         }
         first = false;
       }
       if (!ok) __nanosleep(200000);  // let copies already in flight land before the CTA exits
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
-      auto issue_qk = [&](int t, uint32_t k_smem) {
-        const uint32_t q_smem = sQ + t * C::Q_BYTES;
-#pragma unroll
-        for (int s = 0; s < DQK / C::MMA_K; ++s) {
-          const int e0 = s * C::MMA_K;
-          const uint32_t off = (e0 / C::CHUNK_ELEMS) * C::CHUNK_BYTES + (e0 % C::CHUNK_ELEMS) * C::ESZ;
-          const uint64_t ad = sdesc_sw128(q_smem + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(k_smem + off, 16, 1024);
-          mma_ss<FP8>(tmem + t * 128, ad, bd, C::IDESC_QK, s > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int t, uint32_t v_smem, bool accumulate) {
-#pragma unroll
-        for (int s = 0; s < kBN / C::MMA_K; ++s) {
-          const uint64_t bd = sdesc_sw128(v_smem + s * C::MMA_K * 128, C::CHUNK_BYTES, 1024);
-          const uint32_t a_t = tmem + t * 128 + s * (C::MMA_K * C::ESZ / 4);
-          mma_ts<FP8>(tmem + 256 + t * 128, a_t, bd, C::IDESC_PV, (accumulate || s > 0) ? 1u : 0u);
-        }
-      };
-
-      uint32_t kv_it = 0, q_par = 0;
-      uint32_t p_par[2] = {0, 0}, oe_par[2] = {0, 0};
+      // Descriptor low words of every buffer, computed once; an MMA along K adds
+      // (byte offset >> 4) to them.
+      const uint32_t q_lo0 = sdesc_lo(sQ, 16);
+      const uint32_t k_lo0 = sdesc_lo(sK, 16);
+      const uint32_t v_lo0 = sdesc_lo(sV, C::CHUNK_BYTES);
+      const uint32_t p_lo0 = sdesc_lo(sP, 16);
+      uint32_t gb[2] = {0, 0};  // key blocks tile t has processed in earlier units
+      uint32_t q_par = 0;
+      uint32_t oe_par[2] = {0, 0};
       bool first = true, ok = true;
+      // QK^T for tile t into S_t from K slot s.
+      auto issue_qk = [&](int t, uint32_t s) {
+        const uint32_t a_lo = q_lo0 + t * (C::Q_BYTES >> 4);
+        const uint32_t b_lo = k_lo0 + s * (C::K_BYTES >> 4);
+#pragma unroll
+        for (int kk = 0; kk < DQK / C::MMA_K; ++kk) {
+          const int e0 = kk * C::MMA_K;
+          const uint32_t off = ((e0 / C::CHUNK_ELEMS) * C::CHUNK_BYTES + (e0 % C::CHUNK_ELEMS) * C::ESZ) >> 4;
+          mma_ss_lo<FP8>(tmem + t * 128, a_lo + off, b_lo + off, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t += P V_s, P from shared-memory buffer pbuf (PS) or from S_t in TMEM.
+      auto issue_pv = [&](int t, uint32_t pbuf, uint32_t s, bool accumulate) {
+        const uint32_t d = tmem + 256 + t * 128;
+        const uint32_t b_lo = v_lo0 + s * (C::V_BYTES >> 4);
+        const uint32_t acc = accumulate ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kBN / C::MMA_K; ++kk) {
+          const uint32_t b_off = (kk * C::MMA_K * 128) >> 4;
+          if constexpr (C::PS) {
+            const int e0 = kk * C::MMA_K;
+            const uint32_t off = ((e0 / C::CHUNK_ELEMS) * C::CHUNK_BYTES + (e0 % C::CHUNK_ELEMS) * C::ESZ) >> 4;
+            mma_ss_lo<FP8>(d, p_lo0 + pbuf * (C::P_BYTES >> 4) + off, b_lo + b_off, C::IDESC_PV, kk > 0 ? 1u : acc);
+          } else {
+            mma_ts_lo<FP8>(d, tmem + t * 128 + kk * (C::MMA_K * C::ESZ / 4), b_lo + b_off, C::IDESC_PV,
+                           kk > 0 ? 1u : acc);
+          }
+        }
+      };
+      uint32_t kit = 0, vit = 0;  // K and V ring positions
+      auto take = [&](uint32_t bFull, int nslot, uint32_t& itr, uint32_t& s) -> bool {
+        s = itr % nslot;
+        const bool r = mbar_wait(bFull + 8 * s, (itr / nslot) & 1, abort_flag);
+        ++itr;
+        return r;
+      };
       for (int k = 0; ok; ++k) {
         const int u = unit_for(k, blockIdx.x, gridDim.x);
         if (u >= p.n_units) break;
         const Unit x = decode_unit(u, p);
-        ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
-        if (!ok) break;
-        q_par ^= 1;
-        // block 0: S_0 and S_1 from K_0
-        uint32_t ks = kv_it % C::STAGES;
-        ok = mbar_wait(bKVFull + 8 * ks, (kv_it / C::STAGES) & 1, abort_flag);
-        if (!ok) break;
-        ++kv_it;
-        tc_fence_after();
-        issue_qk(0, sRing + ks * C::STAGE_BYTES);
-        tc_commit(bSFull);
-        if (x.n0 == 1) tc_commit(bQEmpty);
-        issue_qk(1, sRing + ks * C::STAGE_BYTES);
-        tc_commit(bSFull + 8);
-        if (x.n1 == 1) tc_commit(bQEmpty + 8);
-        tc_commit(bKVEmpty + 8 * ks);
-
-        for (int i = 1; i <= x.n1; ++i) {
-          // V_{i-1}
-          const uint32_t vs = kv_it % C::STAGES;
-          ok = mbar_wait(bKVFull + 8 * vs, (kv_it / C::STAGES) & 1, abort_flag);
-          if (!ok) break;
-          ++kv_it;
-          const uint32_t v_smem = sRing + vs * C::STAGE_BYTES;
-          // tile 0: O_0 += P_0,i-1 V_{i-1}
-          if (i - 1 < x.n0) {
-            ok = mbar_wait(bPFull, p_par[0], abort_flag);
+        if constexpr (C::PS) {
+          // Split by role. Warp 1: S_t(j) = Q_t K_j^T once the softmax has copied
+          // S_t's previous block to registers. Warp 2: O_t += P_t(j) V_j once the
+          // softmax has written P_t(j) (and rescaled O_t).
+          if (warp == 1) {
+            ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
             if (!ok) break;
-            p_par[0] ^= 1;
-            if (i == 1 && !first) {
-              ok = mbar_wait(bOEmpty, oe_par[0], abort_flag);
+            q_par ^= 1;
+            for (int j = 0; j < x.n1 && ok; ++j) {
+              uint32_t s;
+              if (!(ok = take(bKFull, C::SK, kit, s))) break;
+              for (int t = 0; t < 2; ++t) {
+                const int n_t = t ? x.n1 : x.n0;
+                if (j >= n_t) continue;
+                const uint32_t gprev = gb[t] + j;  // blocks tile t had before this one
+                if (gprev > 0 && !(ok = mbar_wait(bSFree + 8 * t, (gprev - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                issue_qk(t, s);
+                tc_commit(bSFull + 8 * t);
+                if (j == n_t - 1) tc_commit(bQEmpty + 8 * t);
+              }
               if (!ok) break;
-              oe_par[0] ^= 1;
+              tc_commit(bKEmpty + 8 * s);
             }
-            tc_fence_after();
-            issue_pv(0, v_smem, i > 1);
-            if (i == x.n0) tc_commit(bOFull);
+          } else {
+            for (int j = 0; j < x.n1 && ok; ++j) {
+              uint32_t s;
+              if (!(ok = take(bVFull, C::SV, vit, s))) break;
+              for (int t = 0; t < 2; ++t) {
+                const int n_t = t ? x.n1 : x.n0;
+                if (j >= n_t) continue;
+                const uint32_t g = gb[t] + j;
+                const uint32_t pb = g % C::PBX;
+                ok = mbar_wait(bPFull + 8 * (t * C::PBX + pb), (g / C::PBX) & 1, abort_flag);
+                if (ok && j == 0 && !first) {
+                  ok = mbar_wait(bOEmpty + 8 * t, oe_par[t], abort_flag);
+                  oe_par[t] ^= 1;
+                }
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(t, t * C::PB + pb, s, j > 0);
+                tc_commit(bPDone + 8 * (t * C::PBX + pb));
+                if (j == n_t - 1) tc_commit(bOFull + 8 * t);
+              }
+              if (!ok) break;
+              tc_commit(bVEmpty + 8 * s);
+            }
           }
-          // K_i
-          const bool has_k = i < x.n1;
-          uint32_t ks2 = 0;
-          if (has_k) {
-            ks2 = kv_it % C::STAGES;
-            ok = mbar_wait(bKVFull + 8 * ks2, (kv_it / C::STAGES) & 1, abort_flag);
-            if (!ok) break;
-            ++kv_it;
-            tc_fence_after();
-          }
-          const uint32_t k_smem = sRing + ks2 * C::STAGE_BYTES;
-          if (i < x.n0) {
-            issue_qk(0, k_smem);
-            tc_commit(bSFull);
-            if (i == x.n0 - 1) tc_commit(bQEmpty);
-          }
-          // tile 1: O_1 += P_1,i-1 V_{i-1}
-          ok = mbar_wait(bPFull + 8, p_par[1], abort_flag);
+        } else {
+          // One issuer (warp 1) for both tiles, in the order PV_0(j-1), S_0(j),
+          // PV_1(j-1), S_1(j). The tensor core runs one thread's MMAs in issue
+          // order, so PV_t(j-1) has read P (in S_t's columns) before S_t(j)
+          // overwrites them, and each tile's PV and next QK^T run back to back.
+          if (warp != 1) break;
+          ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
           if (!ok) break;
-          p_par[1] ^= 1;
-          if (i == 1 && !first) {
-            ok = mbar_wait(bOEmpty + 8, oe_par[1], abort_flag);
-            if (!ok) break;
-            oe_par[1] ^= 1;
-          }
+          q_par ^= 1;
+          uint32_t ks;
+          if (!(ok = take(bKFull, C::SK, kit, ks))) break;
           tc_fence_after();
-          issue_pv(1, v_smem, i > 1);
-          if (i == x.n1) tc_commit(bOFull + 8);
-          tc_commit(bKVEmpty + 8 * vs);
-          if (has_k) {
-            issue_qk(1, k_smem);
-            tc_commit(bSFull + 8);
-            if (i == x.n1 - 1) tc_commit(bQEmpty + 8);
-            tc_commit(bKVEmpty + 8 * ks2);
+          for (int t = 0; t < 2; ++t) {
+            issue_qk(t, ks);
+            tc_commit(bSFull + 8 * t);
+            if ((t ? x.n1 : x.n0) == 1) tc_commit(bQEmpty + 8 * t);
+          }
+          tc_commit(bKEmpty + 8 * ks);
+          for (int i = 1; i <= x.n1 && ok; ++i) {
+            uint32_t vs;
+            if (!(ok = take(bVFull, C::SV, vit, vs))) break;
+            const bool has_k = i < x.n1;
+            for (int t = 0; t < 2; ++t) {
+              const int n_t = t ? x.n1 : x.n0;
+              if (i - 1 < n_t) {
+                ok = mbar_wait(bPFull + 8 * t, (gb[t] + i - 1) & 1, abort_flag);
+                if (ok && i == 1 && !first) {
+                  ok = mbar_wait(bOEmpty + 8 * t, oe_par[t], abort_flag);
+                  oe_par[t] ^= 1;
+                }
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(t, 0, vs, i > 1);
+                if (i == n_t) tc_commit(bOFull + 8 * t);
+              }
+              if (t == 0 && has_k) {  // K_i, once tile 0's PV is queued
+                if (!(ok = take(bKFull, C::SK, kit, ks))) break;
+                tc_fence_after();
+              }
+              if (i < n_t) {
+                issue_qk(t, ks);
+                tc_commit(bSFull + 8 * t);
+                if (i == n_t - 1) tc_commit(bQEmpty + 8 * t);
+              }
+            }
+            if (!ok) break;
+            tc_commit(bVEmpty + 8 * vs);
+            if (has_k) tc_commit(bKEmpty + 8 * ks);
           }
         }
+        gb[0] += x.n0;
+        gb[1] += x.n1;
         first = false;
       }
       // Every MMA this thread issued has completed before the CTA frees TMEM.
-      tc_commit(bDrain);
-      if (!mbar_try_wait(bDrain, 0)) {
+      const uint32_t drain = bDrain + 8 * (warp - 1);
+      tc_commit(drain);
+      if (!mbar_try_wait(drain, 0)) {
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bDrain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
     }
@@ -410,9 +498,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem + lane_off + t * 128;
     const uint32_t tO = tmem + lane_off + 256 + t * 128;
-    const uint32_t bS = bSFull + 8 * t, bP = bPFull + 8 * t;
+    const uint32_t bS = bSFull + 8 * t;
     const uint32_t bOf = bOFull + 8 * t, bOe = bOEmpty + 8 * t;
+    // this row's 128-byte lines in the P tiles (PS); 16-byte group c sits at c ^ (r & 7)
+    const uint32_t p_row = sP + t * C::PB * C::P_BYTES + r * 128;
+    const uint32_t p_swz = static_cast<uint32_t>(r & 7);
     uint32_t s_par = 0, o_par = 0;
+    uint32_t g = 0;  // key blocks this warpgroup has finished (PS buffer and parity index)
     bool ok = true;
 
     for (int k = 0; ok; ++k) {
@@ -444,7 +536,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       float m_run = -INFINITY, l_run = 0.0f;
 
-      for (int i = 0; i < n_t; ++i) {
+      for (int i = 0; i < n_t; ++i, ++g) {
         ok = __all_sync(0xffffffffu, mbar_wait(bS, s_par, abort_flag));
         if (!ok) break;
         s_par ^= 1;
@@ -459,6 +551,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         reg_fence32(sr + 32);
         reg_fence32(sr + 64);
         reg_fence32(sr + 96);
+        if constexpr (C::PS) {
+          tc_fence_before();
+          mbar_arrive(bSFree + 8 * t);  // S_t may take the next block now
+        }
 
         const int kv0 = i * kBN;
         if (p.causal) {
@@ -501,6 +597,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             lr = log2f(sv / v_mult);
           }
+          c_blk = fmaxf(c_blk, 1e-30f);  // scales are positive; a zero scale behaves as a tiny one
         }
         const float m_new = fmaxf(m_run, mx * c_blk);
         const bool need_m = m_new > m_run + C::T_LAG;
@@ -517,33 +614,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float l_blk;
         if constexpr (!FP8) {
           const float nm = C::E_SHIFT - m_run;
-          float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
 #pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), c_log2, nm));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), c_log2, nm));
-            sum[(c >> 1) & 7] += p0 + p1;
+          for (int c = 0; c < 128; c += 4) {
+            float x0, x1, x2, x3;
+            ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), c_log2, nm, x0, x1);
+            ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), c_log2, nm, x2, x3);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+            if ((c & 4) == 0) {
+              fadd2(sa, sb, p0, p1);
+              fadd2(sc, sd, p2, p3);
+            } else {
+              fadd2(sc, sd, p0, p1);
+              fadd2(sa, sb, p2, p3);
+            }
             sr[c >> 1] = pack_bf16x2(p0, p1);
+            sr[(c >> 1) + 1] = pack_bf16x2(p2, p3);
           }
-          tmem_st32(tS + 0, sr);
-          tmem_st32(tS + 32, sr + 32);
-          l_blk = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+          l_blk = (sa + sb) + (sc + sd);
         } else {
           // acc: f16x2 partial sums of decode(code)/256 (8 adds per accumulator per block)
           uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
           if constexpr (LEANP) {
-            // w = clamp((8 (c*S - m_run + E + lr) + 56) / 126, 0, 1); code = round(126 w)
+            // w = (8 (c*S - m_run + E + lr) + 56) / 126, clamped below at 0; code = round(126 w)
             const float A = c_blk * (8.0f / 126.0f);
             const float Bc = (8.0f * (C::E_SHIFT - m_run + lr) + 56.0f) * (1.0f / 126.0f);
 #pragma unroll
             for (int c = 0; c < 128; c += 4) {
-              const float w0 = fma_sat(__uint_as_float(sr[c]), A, Bc);
-              const float w1 = fma_sat(__uint_as_float(sr[c + 1]), A, Bc);
-              const float w2 = fma_sat(__uint_as_float(sr[c + 2]), A, Bc);
-              const float w3 = fma_sat(__uint_as_float(sr[c + 3]), A, Bc);
+              float w0, w1, w2, w3;
+              ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), A, Bc, w0, w1);
+              ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), A, Bc, w2, w3);
               // f16 lanes 1536 + code: bits 0x6600 + code
-              const uint32_t u01 = hfma2(pack_f16x2(w0, w1), 0x57E057E0u /*126*/, 0x66006600u /*1536*/);
-              const uint32_t u23 = hfma2(pack_f16x2(w2, w3), 0x57E057E0u, 0x66006600u);
+              const uint32_t u01 = hfma2(pack_f16x2_relu(w0, w1), 0x57E057E0u /*126*/, 0x66006600u /*1536*/);
+              const uint32_t u23 = hfma2(pack_f16x2_relu(w2, w3), 0x57E057E0u, 0x66006600u);
               const int jj = (c >> 1) & 7;
               // (u - 0x66006600) * 128: each lane becomes code << 7
               acc[jj] = hadd2(acc[jj], u01 * 128u + 0xFFCD0000u);
@@ -554,10 +658,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float nm = C::E_SHIFT - m_run + lr;
 #pragma unroll
             for (int c = 0; c < 128; c += 4) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), c_blk, nm));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), c_blk, nm));
-              const float p2 = ex2_approx(fmaf(__uint_as_float(sr[c + 2]), c_blk, nm));
-              const float p3 = ex2_approx(fmaf(__uint_as_float(sr[c + 3]), c_blk, nm));
+              float x0, x1, x2, x3;
+              ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), c_blk, nm, x0, x1);
+              ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), c_blk, nm, x2, x3);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
               const uint32_t w = static_cast<uint32_t>(pack_e4m3x2(p0, p1)) |
                                  (static_cast<uint32_t>(pack_e4m3x2(p2, p3)) << 16);
               const int jj = (c >> 1) & 7;
@@ -566,7 +671,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               sr[c >> 2] = w;
             }
           }
-          tmem_st32(tS + 0, sr);
           const float s01 = f16x2_sum_f32(acc[0]) + f16x2_sum_f32(acc[1]);
           const float s23 = f16x2_sum_f32(acc[2]) + f16x2_sum_f32(acc[3]);
           const float s45 = f16x2_sum_f32(acc[4]) + f16x2_sum_f32(acc[5]);
@@ -576,21 +680,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         l_run += l_blk;
 
-        // rescale this tile's O accumulator (PV_t,i-1 has completed: its commit preceded S_t,i)
-        if (i > 0 && __any_sync(0xffffffffu, need)) {
+        bool rescaled = false;
+        if constexpr (C::PS) {
+          // P buffer g % PB is free once PV of block g-PB has completed; O may be
+          // rescaled once PV of block g-1 (this unit's previous block) has.
+          const uint32_t pb = g % C::PB;
+          bool w_ok = g < static_cast<uint32_t>(C::PB) ||
+                      mbar_wait(bPDone + 8 * (t * C::PBX + pb), ((g / C::PB) - 1) & 1, abort_flag);
+          const bool resc = i > 0 && __any_sync(0xffffffffu, need);
+          if (resc && C::PB > 1)
+            w_ok = w_ok && mbar_wait(bPDone + 8 * (t * C::PBX + (g - 1) % C::PB), ((g - 1) / C::PB) & 1, abort_flag);
+          ok = __all_sync(0xffffffffu, w_ok);
+          if (!ok) break;
+          if (resc) {
+            tc_fence_after();
 #pragma unroll 1
-          for (int cc = 0; cc < DV; cc += 32) {
-            uint32_t orr[32];
-            tmem_ld32(tO + cc, orr);
-            tmem_ld_wait32(orr);
+            for (int cc = 0; cc < DV; cc += 32) {
+              uint32_t orr[32];
+              tmem_ld32(tO + cc, orr);
+              tmem_ld_wait32(orr);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
-            tmem_st32(tO + cc, orr);
+              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+              tmem_st32(tO + cc, orr);
+            }
+            rescaled = true;
           }
+          // P row -> shared memory, 16 bytes at a time, 128-byte swizzle
+          const uint32_t prow = p_row + pb * C::P_BYTES;
+#pragma unroll
+          for (int c = 0; c < 8 * C::P_CHUNKS; ++c)
+            st_shared_v4(prow + (c >> 3) * C::CHUNK_BYTES + (((c & 7) ^ p_swz) << 4), sr[4 * c], sr[4 * c + 1],
+                         sr[4 * c + 2], sr[4 * c + 3]);
+          fence_proxy_async_smem();
+        } else {
+          // rescale this tile's O accumulator (PV_t,i-1 has completed: S_t,i was issued after it)
+          if (i > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+            for (int cc = 0; cc < DV; cc += 32) {
+              uint32_t orr[32];
+              tmem_ld32(tO + cc, orr);
+              tmem_ld_wait32(orr);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+              tmem_st32(tO + cc, orr);
+            }
+          }
+          if constexpr (FP8) {
+            tmem_st32(tS + 0, sr);
+          } else {
+            tmem_st32(tS + 0, sr);
+            tmem_st32(tS + 32, sr + 32);
+          }
+          rescaled = true;
         }
-        tmem_st_wait();
+        if (rescaled) tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bP);
+        mbar_arrive(bPFull + 8 * (t * C::PBX + g % C::PBX));
       }
       if (!ok) break;
 
