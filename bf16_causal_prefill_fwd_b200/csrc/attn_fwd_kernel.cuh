@@ -17,33 +17,32 @@
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer of Q tiles and of the K ring
-//   warps 1, 2  MMA issuers (one thread each; warp 2 only with P in shared
-//               memory), see below
+//   warps 1, 2  MMA issuers (one thread each; warp 2 only with SHARED_S),
+//               see below
 //   warp 3      TMA producer of the V ring
 //   warps 4-7   softmax + epilogue for tile 0 (one thread per query row)
 //   warps 8-11  softmax + epilogue for tile 1
-// With P in shared memory two MMA issuers split by role (warp 1 all QK^T, warp
-// 2 all PV): they wait on different events (scores consumed, probabilities
-// ready), so neither holds up the other's MMAs, and the tensor core runs what
-// both have queued. With P in TMEM, warp 1 alone issues both tiles' MMAs,
-// each tile's PV followed by its next QK^T.
 // The two softmax warpgroups work side by side the way the pages' two-wave
 // ping-pong does ("ZYFA 如何工作？", 双波乒乓调度): while one computes
 // probabilities the tensor core runs the other tile's matrix products. On
 // sm_100 MMA completion is tracked in hardware (tcgen05.commit -> mbarrier),
 // so the overlap needs no instruction-order scheduling.
 //
-// Tensor memory (512 columns x 128 lanes, fp32): [0,128) S_0, [128,256) S_1,
-// [256,384) O_0, [384,512) O_1.
-//
-// Where the probabilities P go (template switch PS):
-//  * PS (FP8): P is written to shared memory in the 128-byte-swizzled K-major
-//    layout the tensor core reads, and PV takes both operands from shared
-//    memory. The softmax frees S_t as soon as it has copied the scores into
-//    registers, so S_t for the next key block is computed while the
-//    probabilities of this block are still being formed.
-//  * otherwise (BF16): P is written over the first columns of S_t in TMEM and
-//    PV reads it from there; S_t for the next block starts once PV_t has read P.
+// Tensor memory (512 columns x 128 lanes, fp32 cells), two layouts (template
+// switch SHARED_S):
+//  * SHARED_S (default): [0,128) one S buffer used by both tiles in turn,
+//    [128,256) O_0, [256,384) O_1, [384,512) P buffers (per tile: two of 32
+//    columns for e4m3, one of 64 for bf16). The softmax releases S as soon as
+//    it has copied the scores to registers, so the tensor core computes the
+//    other tile's S while this tile's probabilities are being formed; P goes
+//    to its own columns and PV reads it there. Two MMA issuers split by role:
+//    warp 1 queues every QK^T (each waits for the previous S to be copied out),
+//    warp 2 every PV (each waits for its P), so neither wait holds up the
+//    other's MMAs.
+//  * otherwise: [0,128) S_0, [128,256) S_1, [256,384) O_0, [384,512) O_1, with
+//    P written over the first columns of S_t; S_t for the next block can only
+//    start after PV_t has read P, so warp 1 alone issues PV_t then QK_t for
+//    each tile in turn (one thread's MMAs run in issue order).
 //
 // Online softmax per row (log2 domain, c = s * log2(e) [* q/k scales]):
 //   m_blk = max_j S_ij; m_new = max(m_run, c * m_blk)
@@ -100,36 +99,36 @@ struct AttnParams {
   float* lse;
 };
 
-template <int DQK, int DV, bool FP8, bool LEANP = false, bool P_SMEM = true>
+template <int DQK, int DV, bool FP8, bool LEANP = false, bool SHARED_S = true>
 struct AttnCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int CHUNK_ELEMS = 128 / ESZ;  // elements in one 128-byte swizzled row
   static constexpr int CHUNK_BYTES = kBM * 128;  // one 128-row x 128-byte swizzle column: 16 KiB
   static constexpr int QK_CHUNKS = (DQK + CHUNK_ELEMS - 1) / CHUNK_ELEMS;
   static constexpr int V_CHUNKS = (DV + CHUNK_ELEMS - 1) / CHUNK_ELEMS;
-  static constexpr int P_CHUNKS = kBN / CHUNK_ELEMS;  // P tile [128 rows, 128 keys]
   static constexpr int Q_BYTES = QK_CHUNKS * CHUNK_BYTES;
   static constexpr int K_BYTES = QK_CHUNKS * CHUNK_BYTES;
   static constexpr int V_BYTES = V_CHUNKS * CHUNK_BYTES;
-  static constexpr int P_BYTES = P_CHUNKS * CHUNK_BYTES;
   static constexpr int STAGE_BYTES = K_BYTES > V_BYTES ? K_BYTES : V_BYTES;
   static constexpr int MMA_K = FP8 ? 32 : 16;  // reduction depth of one tcgen05.mma
-  // P in shared memory (see the file comment); P buffers per tile.
-  static constexpr bool PS = P_SMEM && FP8;
-  static constexpr int PB = PS ? (DQK == 128 ? 2 : 1) : 0;
-  static constexpr int PBX = PS ? PB : 1;  // P-full / P-done barriers per tile
+  // Tensor-memory layout (see the file comment). P columns: bf16 packs 2 keys
+  // per 32-bit column, e4m3 packs 4.
+  static constexpr bool SS = SHARED_S;
+  static constexpr int P_COLS = kBN * ESZ / 4;
+  static constexpr int PB = SS ? (FP8 ? 2 : 1) : 0;  // P buffers per tile
+  static constexpr int PBX = SS ? PB : 1;            // P-full / P-done barriers per tile
+  static constexpr int TM_O = SS ? 128 : 256;        // O_t at TM_O + 128 t
+  static constexpr int TM_P = 384;                   // SS: P(t, b) at TM_P + P_COLS (PB t + b)
   // Separate K and V rings, sized from what shared memory has left.
   static constexpr int SMEM_AVAIL = 227 * 1024 - 2048;  // minus barriers and alignment slack
-  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BYTES - 2 * PB * P_BYTES;
+  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BYTES;
   static constexpr int RING_PAIRS = RING_AVAIL / (K_BYTES + V_BYTES);
   static constexpr int SV = RING_PAIRS >= 2 ? (RING_PAIRS > 4 ? 4 : RING_PAIRS) : 1;
   static constexpr int SK_FIT = (RING_AVAIL - SV * V_BYTES) / K_BYTES;
   static constexpr int SK = SK_FIT > 6 ? 6 : SK_FIT;
   static constexpr int NUM_BARS = 2 + 2 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
-  static constexpr int SMEM_BYTES = 2 * Q_BYTES + 2 * PB * P_BYTES + SK * K_BYTES + SV * V_BYTES +
+  static constexpr int SMEM_BYTES = 2 * Q_BYTES + SK * K_BYTES + SV * V_BYTES +
                                     1024 /*bars*/ + 1024 /*align*/;
-  // P columns in TMEM (non-PS): bf16 packs 2 keys per 32-bit column, e4m3 packs 4.
-  static constexpr int P_COLS = kBN * ESZ / 4;
   static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
   static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
   static_assert(!LEANP || FP8, "Lean P builds e4m3 codes");
@@ -137,6 +136,7 @@ struct AttnCfg {
   static constexpr uint32_t IDESC_PV = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DV, true);
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
   static_assert(SK >= 2 && SV >= 1, "K/V rings");
+  static_assert(!SS || TM_P + 2 * PB * P_COLS <= 512, "TMEM budget");
   static_assert(8 * NUM_BARS + 8 <= 1024, "barrier area");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -194,11 +194,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort_flag);
 }
 
-template <int DQK, int DV, bool FP8, bool LEANP, bool P_SMEM>
+template <int DQK, int DV, bool FP8, bool LEANP, bool SHARED_S>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<DQK, DV, FP8, LEANP, P_SMEM>;
+  using C = AttnCfg<DQK, DV, FP8, LEANP, SHARED_S>;
   extern __shared__ uint8_t smem_raw[];
 
   // 1024-byte aligned base (128-byte swizzle atoms repeat every 1024 bytes).
@@ -207,8 +207,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
 
   const uint32_t sQ = base_u32;                              // 2 query tiles
-  const uint32_t sP = sQ + 2 * C::Q_BYTES;                   // [tile][PB] probability tiles (PS)
-  const uint32_t sK = sP + 2 * C::PB * C::P_BYTES;           // K ring
+  const uint32_t sK = sQ + 2 * C::Q_BYTES;                   // K ring
   const uint32_t sV = sK + C::SK * C::K_BYTES;               // V ring
   const uint32_t sBar = sV + C::SV * C::V_BYTES;
   uint8_t* bar_ptr = base + (sBar - base_u32);
@@ -223,9 +222,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bVFull = bKEmpty + 8 * C::SK;           // [SV] TMA -> PV issuer
   const uint32_t bVEmpty = bVFull + 8 * C::SV;           // [SV] PV issuer -> TMA
   const uint32_t bSFull = bVEmpty + 8 * C::SV;           // [2]  QK issuer -> softmax
-  const uint32_t bSFree = bSFull + 16;                   // [2]  softmax -> QK issuer (128 arrivals; PS)
-  // P full (softmax -> PV issuer, 128 arrivals) and P done (PV issuer -> softmax
-  // and, without PS, -> QK issuer), per tile and P buffer. One barrier per
+  const uint32_t bSFree = bSFull + 16;                   // [1]  softmax -> QK issuer (128 arrivals; SS)
+  // P full (softmax -> PV issuer, 128 arrivals) and P done (PV issuer ->
+  // softmax), per tile and P buffer. One barrier per
   // buffer keeps a softmax that runs a block ahead from completing two phases of
   // the barrier the PV issuer is about to wait on.
   const uint32_t bPFull = bSFree + 16;                   // [2][PBX]
@@ -243,7 +242,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(bQFull + 8 * t, 1);
         mbar_init(bQEmpty + 8 * t, 1);
         mbar_init(bSFull + 8 * t, 1);
-        mbar_init(bSFree + 8 * t, 128);
+        if (t == 0) mbar_init(bSFree, 128);
         for (int b = 0; b < C::PBX; ++b) {
           mbar_init(bPFull + 8 * (t * C::PBX + b), 128);
           mbar_init(bPDone + 8 * (t * C::PBX + b), 1);
@@ -334,7 +333,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t q_lo0 = sdesc_lo(sQ, 16);
       const uint32_t k_lo0 = sdesc_lo(sK, 16);
       const uint32_t v_lo0 = sdesc_lo(sV, C::CHUNK_BYTES);
-      const uint32_t p_lo0 = sdesc_lo(sP, 16);
       uint32_t gb[2] = {0, 0};  // key blocks tile t has processed in earlier units
       uint32_t q_par = 0;
       uint32_t oe_par[2] = {0, 0};
@@ -347,28 +345,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kk = 0; kk < DQK / C::MMA_K; ++kk) {
           const int e0 = kk * C::MMA_K;
           const uint32_t off = ((e0 / C::CHUNK_ELEMS) * C::CHUNK_BYTES + (e0 % C::CHUNK_ELEMS) * C::ESZ) >> 4;
-          mma_ss_lo<FP8>(tmem + t * 128, a_lo + off, b_lo + off, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_ss_lo<FP8>(tmem + (C::SS ? 0 : t * 128), a_lo + off, b_lo + off, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t += P V_s, P from shared-memory buffer pbuf (PS) or from S_t in TMEM.
+      // O_t += P V_s with P from TMEM: buffer pbuf (SS) or the first columns of S_t.
       auto issue_pv = [&](int t, uint32_t pbuf, uint32_t s, bool accumulate) {
-        const uint32_t d = tmem + 256 + t * 128;
+        const uint32_t d = tmem + C::TM_O + t * 128;
         const uint32_t b_lo = v_lo0 + s * (C::V_BYTES >> 4);
+        const uint32_t a_t = tmem + (C::SS ? C::TM_P + pbuf * C::P_COLS : t * 128);
         const uint32_t acc = accumulate ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kBN / C::MMA_K; ++kk) {
-          const uint32_t b_off = (kk * C::MMA_K * 128) >> 4;
-          if constexpr (C::PS) {
-            const int e0 = kk * C::MMA_K;
-            const uint32_t off = ((e0 / C::CHUNK_ELEMS) * C::CHUNK_BYTES + (e0 % C::CHUNK_ELEMS) * C::ESZ) >> 4;
-            mma_ss_lo<FP8>(d, p_lo0 + pbuf * (C::P_BYTES >> 4) + off, b_lo + b_off, C::IDESC_PV, kk > 0 ? 1u : acc);
-          } else {
-            mma_ts_lo<FP8>(d, tmem + t * 128 + kk * (C::MMA_K * C::ESZ / 4), b_lo + b_off, C::IDESC_PV,
-                           kk > 0 ? 1u : acc);
-          }
-        }
+        for (int kk = 0; kk < kBN / C::MMA_K; ++kk)
+          mma_ts_lo<FP8>(d, a_t + kk * (C::MMA_K * C::ESZ / 4), b_lo + ((kk * C::MMA_K * 128) >> 4), C::IDESC_PV,
+                         kk > 0 ? 1u : acc);
       };
       uint32_t kit = 0, vit = 0;  // K and V ring positions
+      uint32_t nq = 0;            // QK^T products issued (SS: uses of the one S buffer)
       auto take = [&](uint32_t bFull, int nslot, uint32_t& itr, uint32_t& s) -> bool {
         s = itr % nslot;
         const bool r = mbar_wait(bFull + 8 * s, (itr / nslot) & 1, abort_flag);
@@ -379,10 +371,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int u = unit_for(k, blockIdx.x, gridDim.x);
         if (u >= p.n_units) break;
         const Unit x = decode_unit(u, p);
-        if constexpr (C::PS) {
-          // Split by role. Warp 1: S_t(j) = Q_t K_j^T once the softmax has copied
-          // S_t's previous block to registers. Warp 2: O_t += P_t(j) V_j once the
-          // softmax has written P_t(j) (and rescaled O_t).
+        if constexpr (C::SS) {
+          // Split by role. Warp 1: S = Q_t K_j^T once the softmax has copied the
+          // previous S out. Warp 2: O_t += P_t(j) V_j once the softmax has written
+          // P_t(j) (and rescaled O_t).
           if (warp == 1) {
             ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
             if (!ok) break;
@@ -393,8 +385,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int t = 0; t < 2; ++t) {
                 const int n_t = t ? x.n1 : x.n0;
                 if (j >= n_t) continue;
-                const uint32_t gprev = gb[t] + j;  // blocks tile t had before this one
-                if (gprev > 0 && !(ok = mbar_wait(bSFree + 8 * t, (gprev - 1) & 1, abort_flag))) break;
+                if (nq > 0 && !(ok = mbar_wait(bSFree, (nq - 1) & 1, abort_flag))) break;
+                ++nq;
                 tc_fence_after();
                 issue_qk(t, s);
                 tc_commit(bSFull + 8 * t);
@@ -496,15 +488,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int t = (warp - 4) >> 2;            // query tile of this warpgroup
     const int r = threadIdx.x - 128 - 128 * t;  // row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128;
-    const uint32_t tO = tmem + lane_off + 256 + t * 128;
+    const uint32_t tS = tmem + lane_off + (C::SS ? 0 : t * 128);
+    const uint32_t tO = tmem + lane_off + C::TM_O + t * 128;
+    const uint32_t tP = tmem + lane_off + C::TM_P + t * C::PB * C::P_COLS;  // SS
     const uint32_t bS = bSFull + 8 * t;
     const uint32_t bOf = bOFull + 8 * t, bOe = bOEmpty + 8 * t;
-    // this row's 128-byte lines in the P tiles (PS); 16-byte group c sits at c ^ (r & 7)
-    const uint32_t p_row = sP + t * C::PB * C::P_BYTES + r * 128;
-    const uint32_t p_swz = static_cast<uint32_t>(r & 7);
     uint32_t s_par = 0, o_par = 0;
-    uint32_t g = 0;  // key blocks this warpgroup has finished (PS buffer and parity index)
+    uint32_t g = 0;  // key blocks this warpgroup has finished (SS buffer and parity index)
     bool ok = true;
 
     for (int k = 0; ok; ++k) {
@@ -551,9 +541,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         reg_fence32(sr + 32);
         reg_fence32(sr + 64);
         reg_fence32(sr + 96);
-        if constexpr (C::PS) {
+        if constexpr (C::SS) {
           tc_fence_before();
-          mbar_arrive(bSFree + 8 * t);  // S_t may take the next block now
+          mbar_arrive(bSFree);  // S may take the next product now
         }
 
         const int kv0 = i * kBN;
@@ -680,8 +670,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         l_run += l_blk;
 
-        bool rescaled = false;
-        if constexpr (C::PS) {
+        if constexpr (C::SS) {
           // P buffer g % PB is free once PV of block g-PB has completed; O may be
           // rescaled once PV of block g-1 (this unit's previous block) has.
           const uint32_t pb = g % C::PB;
@@ -692,8 +681,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             w_ok = w_ok && mbar_wait(bPDone + 8 * (t * C::PBX + (g - 1) % C::PB), ((g - 1) / C::PB) & 1, abort_flag);
           ok = __all_sync(0xffffffffu, w_ok);
           if (!ok) break;
+          tc_fence_after();
           if (resc) {
-            tc_fence_after();
 #pragma unroll 1
             for (int cc = 0; cc < DV; cc += 32) {
               uint32_t orr[32];
@@ -703,15 +692,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
               tmem_st32(tO + cc, orr);
             }
-            rescaled = true;
           }
-          // P row -> shared memory, 16 bytes at a time, 128-byte swizzle
-          const uint32_t prow = p_row + pb * C::P_BYTES;
-#pragma unroll
-          for (int c = 0; c < 8 * C::P_CHUNKS; ++c)
-            st_shared_v4(prow + (c >> 3) * C::CHUNK_BYTES + (((c & 7) ^ p_swz) << 4), sr[4 * c], sr[4 * c + 1],
-                         sr[4 * c + 2], sr[4 * c + 3]);
-          fence_proxy_async_smem();
+          // P row -> its own TMEM columns
+          tmem_st32(tP + pb * C::P_COLS, sr);
+          if constexpr (!FP8) tmem_st32(tP + pb * C::P_COLS + 32, sr + 32);
         } else {
           // rescale this tile's O accumulator (PV_t,i-1 has completed: S_t,i was issued after it)
           if (i > 0 && __any_sync(0xffffffffu, need)) {
@@ -731,9 +715,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tS + 0, sr);
             tmem_st32(tS + 32, sr + 32);
           }
-          rescaled = true;
         }
-        if (rescaled) tmem_st_wait();
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bPFull + 8 * (t * C::PBX + g % C::PBX));
       }

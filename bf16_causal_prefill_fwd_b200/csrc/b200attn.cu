@@ -76,15 +76,15 @@ int device_ok(int* sm_count) {
   return B200ATTN_OK;
 }
 
-template <int DQK, int DV, bool FP8, bool LEANP, bool P_SMEM>
+template <int DQK, int DV, bool FP8, bool LEANP, bool SHARED_S>
 int launch_attn_t(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
-  using C = AttnCfg<DQK, DV, FP8, LEANP, P_SMEM>;
+  using C = AttnCfg<DQK, DV, FP8, LEANP, SHARED_S>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, FP8, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, FP8, d_qk, p.Hkv, p.N, p.B) ||
       !make_tmap(&tv, v, FP8, d_v, p.Hkv, p.N, p.B))
     return B200ATTN_ERR_CUDA;
-  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, LEANP, P_SMEM>;
+  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, LEANP, SHARED_S>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
@@ -92,17 +92,19 @@ int launch_attn_t(const void* q, const void* k, const void* v, const AttnParams&
   return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
 }
 
-// Where the probabilities go: shared memory (default) or tensor memory.
-// B200ATTN_P_SMEM=0 selects the latter; read on every call so A/B runs need no rebuild.
-bool p_in_smem() {
-  const char* e = std::getenv("B200ATTN_P_SMEM");
+// Tensor-memory layout of the attention kernel: one S buffer shared by both
+// query tiles (default) or one per tile with P written over it.
+// B200ATTN_SHARED_S=0 selects the latter; read on every call so A/B runs need
+// no rebuild.
+bool shared_s() {
+  const char* e = std::getenv("B200ATTN_SHARED_S");
   return !(e && std::strcmp(e, "0") == 0);
 }
 
 template <int DQK, int DV, bool FP8, bool LEANP = false>
 int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
-  if (p_in_smem()) return launch_attn_t<DQK, DV, FP8, LEANP, true>(q, k, v, p, d_qk, d_v, sm_count, stream);
+  if (shared_s()) return launch_attn_t<DQK, DV, FP8, LEANP, true>(q, k, v, p, d_qk, d_v, sm_count, stream);
   return launch_attn_t<DQK, DV, FP8, LEANP, false>(q, k, v, p, d_qk, d_v, sm_count, stream);
 }
 
