@@ -30,9 +30,15 @@
 //
 // Tensor memory (512 columns x 128 lanes, fp32 cells), two layouts (template
 // switch SHARED_S):
-//  * SHARED_S (default): [0,128) one S buffer used by both tiles in turn,
-//    [128,256) O_0, [256,384) O_1, [384,512) P buffers (per tile: two of 32
-//    columns for e4m3, one of 64 for bf16). The softmax releases S as soon as
+//  * SHARED_S (default): [0,128) one S buffer used by both tiles in turn, then
+//    O_0, O_1 and a P buffer per tile. bf16: O_t at 128 + 128 t, P_t (64
+//    columns) at 384 + 64 t. e4m3: O_t at 128 + 160 t with 144 columns, the
+//    last 16 holding the row sum of the rounded probabilities, which the
+//    tensor core forms by multiplying P with a shared-memory tile of ones
+//    placed after V (PV runs with N = 144); P_t (32 columns) at 448 + 32 t.
+//    Row sums by the tensor core are used with per-head scales; with
+//    per-block V scales P carries a per-block factor and the softmax keeps the
+//    sum in registers as in the other layout. The softmax releases S as soon as
 //    it has copied the scores to registers, so the tensor core computes the
 //    other tile's S while this tile's probabilities are being formed; P goes
 //    to its own columns and PV reads it there. Two MMA issuers split by role:
@@ -115,25 +121,33 @@ struct AttnCfg {
   // per 32-bit column, e4m3 packs 4.
   static constexpr bool SS = SHARED_S;
   static constexpr int P_COLS = kBN * ESZ / 4;
-  static constexpr int PB = SS ? (FP8 ? 2 : 1) : 0;  // P buffers per tile
+  // RS: the tensor core forms the row sums of the rounded e4m3 probabilities.
+  // PV runs with N = d_v + 16, the extra B columns reading a shared-memory tile
+  // of ones, so columns d_v.. of O_t accumulate sum_j P_ij with the same
+  // rescales as O.
+  static constexpr bool RS = SS && FP8;
+  static constexpr int DVX = DV + (RS ? 16 : 0);     // O_t columns (output, then row sum)
+  static constexpr int PB = SS ? (FP8 && !RS ? 2 : 1) : 0;  // P buffers per tile
   static constexpr int PBX = SS ? PB : 1;            // P-full / P-done barriers per tile
-  static constexpr int TM_O = SS ? 128 : 256;        // O_t at TM_O + 128 t
-  static constexpr int TM_P = 384;                   // SS: P(t, b) at TM_P + P_COLS (PB t + b)
+  static constexpr int O_STRIDE = (DVX + 31) / 32 * 32;  // TMEM columns per O_t, kept 32-aligned
+  static constexpr int TM_O = SS ? 128 : 256;        // O_t at TM_O + O_STRIDE t
+  static constexpr int TM_P = SS ? 128 + 2 * O_STRIDE : 384;  // SS: P(t, b) at TM_P + P_COLS (PB t + b)
+  static constexpr int ONES_BYTES = RS ? CHUNK_BYTES : 0;
   // Separate K and V rings, sized from what shared memory has left.
   static constexpr int SMEM_AVAIL = 227 * 1024 - 2048;  // minus barriers and alignment slack
-  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BYTES;
+  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BYTES - ONES_BYTES;
   static constexpr int RING_PAIRS = RING_AVAIL / (K_BYTES + V_BYTES);
   static constexpr int SV = RING_PAIRS >= 2 ? (RING_PAIRS > 4 ? 4 : RING_PAIRS) : 1;
   static constexpr int SK_FIT = (RING_AVAIL - SV * V_BYTES) / K_BYTES;
   static constexpr int SK = SK_FIT > 6 ? 6 : SK_FIT;
   static constexpr int NUM_BARS = 2 + 2 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
-  static constexpr int SMEM_BYTES = 2 * Q_BYTES + SK * K_BYTES + SV * V_BYTES +
+  static constexpr int SMEM_BYTES = 2 * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES +
                                     1024 /*bars*/ + 1024 /*align*/;
   static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
   static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
   static_assert(!LEANP || FP8, "Lean P builds e4m3 codes");
   static constexpr uint32_t IDESC_QK = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, kBN, false);
-  static constexpr uint32_t IDESC_PV = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DV, true);
+  static constexpr uint32_t IDESC_PV = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DVX, true);
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
   static_assert(SK >= 2 && SV >= 1, "K/V rings");
   static_assert(!SS || TM_P + 2 * PB * P_COLS <= 512, "TMEM budget");
@@ -209,7 +223,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sQ = base_u32;                              // 2 query tiles
   const uint32_t sK = sQ + 2 * C::Q_BYTES;                   // K ring
   const uint32_t sV = sK + C::SK * C::K_BYTES;               // V ring
-  const uint32_t sBar = sV + C::SV * C::V_BYTES;
+  const uint32_t sOnes = sV + C::SV * C::V_BYTES;          // RS: e4m3 ones, B columns d_v..d_v+15
+  const uint32_t sBar = sOnes + C::ONES_BYTES;
   uint8_t* bar_ptr = base + (sBar - base_u32);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NUM_BARS + 4);
@@ -268,6 +283,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
     tmem_alloc(smem_addr(tmem_slot), 512);
     tmem_relinquish();
+  }
+  if constexpr (C::RS) {
+    // e4m3 1.0 is 0x38 in every byte, so the swizzle pattern does not matter
+    for (int i = threadIdx.x; i < C::ONES_BYTES / 16; i += kAttnThreads)
+      st_shared_v4(sOnes + 16 * i, 0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -349,9 +370,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       };
       // O_t += P V_s with P from TMEM: buffer pbuf (SS) or the first columns of S_t.
+      // RS: the second 128-byte column block of B (leading byte offset) is the
+      // ones tile, so the row sums land in O_t's extra columns.
       auto issue_pv = [&](int t, uint32_t pbuf, uint32_t s, bool accumulate) {
-        const uint32_t d = tmem + C::TM_O + t * 128;
-        const uint32_t b_lo = v_lo0 + s * (C::V_BYTES >> 4);
+        const uint32_t d = tmem + C::TM_O + t * C::O_STRIDE;
+        const uint32_t v_stage = sV + s * C::V_BYTES;
+        const uint32_t b_lo = C::RS ? sdesc_lo(v_stage, sOnes - v_stage) : v_lo0 + s * (C::V_BYTES >> 4);
         const uint32_t a_t = tmem + (C::SS ? C::TM_P + pbuf * C::P_COLS : t * 128);
         const uint32_t acc = accumulate ? 1u : 0u;
 #pragma unroll
@@ -489,7 +513,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int r = threadIdx.x - 128 - 128 * t;  // row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem + lane_off + (C::SS ? 0 : t * 128);
-    const uint32_t tO = tmem + lane_off + C::TM_O + t * 128;
+    const uint32_t tO = tmem + lane_off + C::TM_O + t * C::O_STRIDE;
     const uint32_t tP = tmem + lane_off + C::TM_P + t * C::PB * C::P_COLS;  // SS
     const uint32_t bS = bSFull + 8 * t;
     const uint32_t bOf = bOFull + 8 * t, bOe = bOEmpty + 8 * t;
@@ -525,6 +549,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       float m_run = -INFINITY, l_run = 0.0f;
+      // RS with per-head scales: the row sum comes from O_t's extra columns. With
+      // per-block V scales P carries sv[i] / s_ref, so the sum is kept here instead.
+      const bool mma_sum = C::RS && !p.per_block;
 
       for (int i = 0; i < n_t; ++i, ++g) {
         ok = __all_sync(0xffffffffu, mbar_wait(bS, s_par, abort_flag));
@@ -623,6 +650,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             sr[(c >> 1) + 1] = pack_bf16x2(p2, p3);
           }
           l_blk = (sa + sb) + (sc + sd);
+        } else if (mma_sum) {
+          // codes only; the tensor core adds them up
+          if constexpr (LEANP) {
+            const float A = c_blk * (8.0f / 126.0f);
+            const float Bc = (8.0f * (C::E_SHIFT - m_run + lr) + 56.0f) * (1.0f / 126.0f);
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+              float w0, w1, w2, w3;
+              ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), A, Bc, w0, w1);
+              ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), A, Bc, w2, w3);
+              const uint32_t u01 = hfma2(pack_f16x2_relu(w0, w1), 0x57E057E0u, 0x66006600u);
+              const uint32_t u23 = hfma2(pack_f16x2_relu(w2, w3), 0x57E057E0u, 0x66006600u);
+              sr[c >> 2] = prmt(u01, u23, 0x6420u);
+            }
+          } else {
+            const float nm = C::E_SHIFT - m_run + lr;
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+              float x0, x1, x2, x3;
+              ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), c_blk, nm, x0, x1);
+              ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), c_blk, nm, x2, x3);
+              sr[c >> 2] = static_cast<uint32_t>(pack_e4m3x2(ex2_approx(x0), ex2_approx(x1))) |
+                           (static_cast<uint32_t>(pack_e4m3x2(ex2_approx(x2), ex2_approx(x3))) << 16);
+            }
+          }
+          l_blk = 0.0f;
         } else {
           // acc: f16x2 partial sums of decode(code)/256 (8 adds per accumulator per block)
           uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -692,6 +745,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
               tmem_st32(tO + cc, orr);
             }
+            if constexpr (C::RS) {
+              uint32_t orr[16];
+              tmem_ld16(tO + DV, orr);
+              tmem_ld_wait16(orr);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+              tmem_st16(tO + DV, orr);
+            }
           }
           // P row -> its own TMEM columns
           tmem_st32(tP + pb * C::P_COLS, sr);
@@ -727,6 +788,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) break;
       o_par ^= 1;
       tc_fence_after();
+      if (mma_sum) {
+        uint32_t lr16[16];
+        tmem_ld16(tO + DV, lr16);
+        tmem_ld_wait16(lr16);
+        l_run = __uint_as_float(lr16[0]);
+      }
       const float inv_l = v_mult / l_run;
       const bool row_ok = qrow < p.N;
       __nv_bfloat16* orow = p.o + ((static_cast<size_t>(x.b) * p.N + (row_ok ? qrow : 0)) * p.Hq + x.hq) * DV;

@@ -134,8 +134,18 @@ def test_fp8_per_block_scales_match_oracle(shape, causal, fp8_p):
     check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
 
 
-def test_fp8_per_block_equals_per_head_when_scales_agree():
-    """Per-block scales that all equal the per-head scale give bitwise the same output."""
+# Per-head and per-block runs form the same e4m3 probabilities when the scales
+# agree, but may add them up in different units: with per-head scales the
+# tensor core sums the rounded probabilities in fp32, with per-block scales the
+# softmax threads sum them in f16 pairs (8 additions per accumulator and block,
+# each rounding by at most 2^-11 of the partial sum) before widening to fp32.
+# The row sums, and so the outputs, may differ by up to about 8 * 2^-11.
+ROW_SUM_UNIT_TOL = 8 * 2.0 ** -11
+
+
+def test_fp8_per_block_matches_per_head_when_scales_agree():
+    """Per-block scales that all equal the per-head scale give the per-head output
+    up to the rounding of the row sum."""
     q, k, v = workloads.draw(workloads.gaussian(1, 4, 2, 384, 128, 128, seed=9))
     codes, _ = oracle_fp8_inputs(q, k, v, granularity="head")
     q8, sq, k8, sk, v8, sv = to_gpu_fp8(codes)
@@ -143,7 +153,10 @@ def test_fp8_per_block_equals_per_head_when_scales_agree():
     rep = lambda s: s[:, :, None].expand(-1, -1, 3).contiguous()
     o_blk = b2.attn_fwd(q8, k8, v8, q_scale=rep(sq), k_scale=rep(sk), v_scale=rep(sv), scale_granularity="block")
     assert b2.check() == 0
-    assert torch.equal(o_head, o_blk)
+    a, b = f32(o_head), f32(o_blk)
+    assert oracle.rel_rms(b, a) <= ROW_SUM_UNIT_TOL
+    # elementwise: the same row-sum factor plus one bf16 rounding of the output
+    assert np.all(np.abs(b - a) <= (ROW_SUM_UNIT_TOL + 2.0 ** -7) * np.abs(a) + 1e-6)
 
 
 @pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
