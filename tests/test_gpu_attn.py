@@ -57,6 +57,23 @@ SMALL = [
 FP8_P = ["lean", "mufu"]
 
 
+# FP8 with per-head scales has two kernels: two query tiles per CTA (default)
+# and one tile per CTA (B200ATTN_FP8_TILE=1); the tests marked with this
+# fixture run both.
+FP8_KERNELS = ["pair", "tile"]
+
+
+@pytest.fixture
+def fp8_kernel(request):
+    old = os.environ.get("B200ATTN_FP8_TILE")
+    os.environ["B200ATTN_FP8_TILE"] = "1" if request.param == "tile" else "0"
+    yield request.param
+    if old is None:
+        os.environ.pop("B200ATTN_FP8_TILE", None)
+    else:
+        os.environ["B200ATTN_FP8_TILE"] = old
+
+
 @pytest.fixture
 def fp8_p(request):
     old = os.environ.get("B200ATTN_FP8_P")
@@ -95,10 +112,11 @@ def test_bf16_matches_oracle(shape, causal):
     check_lse(lse, ref_lse)
 
 
+@pytest.mark.parametrize("fp8_kernel", FP8_KERNELS, indirect=True)
 @pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
 @pytest.mark.parametrize("shape", SMALL)
 @pytest.mark.parametrize("causal", [True, False])
-def test_fp8_matches_oracle(shape, causal, fp8_p):
+def test_fp8_matches_oracle(shape, causal, fp8_p, fp8_kernel):
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq + 1))
     codes, deq = oracle_fp8_inputs(q, k, v)
@@ -205,10 +223,44 @@ def test_causality_on_gpu():
     assert torch.equal(o1[:, :300], o2[:, :300])
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8-lean", "fp8-mufu"])
+# More units than SMs, so each persistent CTA runs several units back to back
+# (including the one-block units of the first query tile), and the unit-to-unit
+# hand-offs of Q, O and the running max are exercised.
+MANY_UNITS = (4, 32, 8, 1024, 128)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_many_units_per_cta(causal):
+    B, Hq, Hkv, N, dqk = MANY_UNITS
+    q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=21))
+    o, _ = run_bf16(q, k, v, causal=causal)
+    heads = [0, 9, Hq - 1]
+    rows = np.arange(N)
+    ref, _ = oracle_on_sample(q, k, v, heads, rows, causal=causal)
+    err = oracle.rel_rms(gather_sample(o, heads, rows), ref)
+    assert err <= BF16_TOL, err
+
+
+@pytest.mark.parametrize("fp8_kernel", FP8_KERNELS, indirect=True)
+@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_many_units_per_cta(causal, fp8_p, fp8_kernel):
+    B, Hq, Hkv, N, dqk = MANY_UNITS
+    q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=22))
+    codes, deq = oracle_fp8_inputs(q, k, v)
+    o, _ = run_fp8(codes, causal=causal)
+    heads = [0, 9, Hq - 1]
+    rows = np.arange(N)
+    ref, _ = oracle_on_sample(*deq, heads, rows, causal=causal)
+    err = oracle.rel_rms(gather_sample(o, heads, rows), ref)
+    assert err <= FP8_TOL, err
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8-lean", "fp8-mufu", "fp8-lean-tile"])
 def test_bitwise_deterministic_over_1000_launches(dtype, monkeypatch):
     if dtype.startswith("fp8"):
-        monkeypatch.setenv("B200ATTN_FP8_P", dtype[4:])
+        monkeypatch.setenv("B200ATTN_FP8_P", dtype.split("-")[1])
+        monkeypatch.setenv("B200ATTN_FP8_TILE", "1" if dtype.endswith("-tile") else "0")
     q, k, v = workloads.draw(workloads.gaussian(1, 8, 2, 2048, 128, 128, seed=8))
     if dtype == "bf16":
         args = (q.cuda(), k.cuda(), v.cuda())
