@@ -11,6 +11,8 @@ from ._binding import (  # noqa: F401
     check,
     load_library,
     quantize_fp8,
+    quantize_qkv_fp8,
+    quantize_qkv_workspace_bytes,
     quantize_workspace_bytes,
     selftest_wait_timeout,
     version,

@@ -49,6 +49,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.b200attn_quantize_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.b200attn_quantize_fp8.restype = i
     lib.b200attn_quantize_fp8.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
+    lib.b200attn_quantize_qkv_workspace_bytes.restype = sz
+    lib.b200attn_quantize_qkv_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.b200attn_quantize_qkv_fp8.restype = i
+    lib.b200attn_quantize_qkv_fp8.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp]
     lib.b200attn_check.restype = i
     lib.b200attn_check.argtypes = [vp]
     lib.b200attn_strerror.restype = ctypes.c_char_p
@@ -160,6 +164,44 @@ def quantize_fp8(x, *, granularity: str = "head", hadamard: bool = False, out=No
     return out, scale
 
 
+def quantize_qkv_workspace_bytes(B, N, Hq, Hkv, granularity="head") -> int:
+    return int(load_library().b200attn_quantize_qkv_workspace_bytes(B, N, Hq, Hkv, _GRAN[granularity]))
+
+
+def quantize_qkv_fp8(q, k, v, *, granularity: str = "head", hadamard: bool = False, out=None, workspace=None,
+                     stream=None):
+    """bf16 Q, K, V -> (q8, sq, k8, sk, v8, sv) through b200attn_quantize_qkv_fp8: one
+    launch per pass for all three tensors; the rotation (``hadamard``) applies to
+    Q and K only. ``out`` may pass the six output tensors to fill."""
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_cuda_contig(name, t)
+        if t.dtype != torch.bfloat16 or t.dim() != 4:
+            raise ValueError(f"{name} must be bf16 [B, N, H, d]")
+    B, N, Hq, d_qk = q.shape
+    Hkv, d_v = k.shape[2], v.shape[3]
+    if k.shape != (B, N, Hkv, d_qk) or v.shape != (B, N, Hkv, d_v):
+        raise ValueError("shape mismatch between q, k and v")
+    if out is None:
+        nb = math.ceil(N / BLOCK)
+        dev = q.device
+        out = []
+        for t, H in ((q, Hq), (k, Hkv), (v, Hkv)):
+            out.append(torch.empty(t.shape, dtype=torch.float8_e4m3fn, device=dev))
+            out.append(torch.empty((B, H) if granularity == "head" else (B, H, nb), dtype=torch.float32, device=dev))
+    q8, sq, k8, sk, v8, sv = out
+    need = quantize_qkv_workspace_bytes(B, N, Hq, Hkv, granularity)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.b200attn_quantize_qkv_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk),
+                                       _ptr(sv), B, N, Hq, Hkv, d_qk, d_v, _GRAN[granularity],
+                                       1 if hadamard else 0, _ptr(workspace), wbytes, _stream_handle(stream))
+    if rc != 0:
+        raise B200AttnError(rc, "b200attn_quantize_qkv_fp8")
+    return q8, sq, k8, sk, v8, sv
+
+
 def attn_func(q, k, v, softmax_scale: float | None = None, causal: bool = True, *, fp8: bool = False,
               hadamard: bool = False, granularity: str = "head", return_lse: bool = False, stream=None):
     """flash_attn_func-style call on bf16 [B,N,H,d] tensors.
@@ -171,9 +213,7 @@ def attn_func(q, k, v, softmax_scale: float | None = None, causal: bool = True, 
     if not fp8:
         return attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale, return_lse=return_lse,
                         stream=stream)
-    q8, sq = quantize_fp8(q, granularity=granularity, hadamard=hadamard, stream=stream)
-    k8, sk = quantize_fp8(k, granularity=granularity, hadamard=hadamard, stream=stream)
-    v8, sv = quantize_fp8(v, granularity=granularity, hadamard=False, stream=stream)
+    q8, sq, k8, sk, v8, sv = quantize_qkv_fp8(q, k, v, granularity=granularity, hadamard=hadamard, stream=stream)
     return attn_fwd(q8, k8, v8, causal=causal, softmax_scale=softmax_scale, q_scale=sq, k_scale=sk,
                     v_scale=sv, scale_granularity=granularity, return_lse=return_lse, stream=stream)
 

@@ -152,6 +152,18 @@ int launch_quant(const void* x, void* y, float* scale, int B, int N, int H, int 
   return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
 }
 
+template <int DQK, int DV, bool HAD>
+int launch_quant_qkv(const b200::QkvQuant& a, int B, int gran, cudaStream_t stream) {
+  const dim3 grid(a.nblk, a.H[0] + a.H[1] + a.H[2], B);
+  if (gran == B200ATTN_SCALE_PER_HEAD) {
+    b200::quant_qkv_absmax_kernel<DQK, DV, HAD><<<grid, b200::kQuantThreads, 0, stream>>>(a);
+    b200::quant_qkv_encode_kernel<DQK, DV, HAD, true><<<grid, b200::kQuantThreads, 0, stream>>>(a);
+  } else {
+    b200::quant_qkv_encode_kernel<DQK, DV, HAD, false><<<grid, b200::kQuantThreads, 0, stream>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -253,6 +265,72 @@ int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale, int B, int N
   return hadamard ? launch_quant<192, true>(x, x_fp8, scale, B, N, H, granularity, workspace, st)
                   : launch_quant<192, false>(x, x_fp8, scale, B, N, H, granularity, workspace, st);
 }
+
+// ---------------------------------------------------------------------------------------------
+// Q, K and V quantised by one launch per pass.
+// ---------------------------------------------------------------------------------------------
+
+
+size_t b200attn_quantize_qkv_workspace_bytes(int B, int N, int Hq, int Hkv, int granularity) {
+  if (B < 1 || N < 1 || Hq < 1 || Hkv < 1) return 0;
+  if (granularity != B200ATTN_SCALE_PER_HEAD) return 0;
+  const size_t nblk = (static_cast<size_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  return static_cast<size_t>(B) * (static_cast<size_t>(Hq) + 2 * static_cast<size_t>(Hkv)) * nblk * sizeof(float);
+}
+
+int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v, void* q_fp8, void* k_fp8, void* v_fp8,
+                              float* q_scale, float* k_scale, float* v_scale, int B, int N, int Hq, int Hkv,
+                              int d_qk, int d_v, int granularity, int hadamard, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !q_fp8 || !k_fp8 || !v_fp8 || !q_scale || !k_scale || !v_scale) return B200ATTN_ERR_INVALID;
+  if (B < 1 || N < 1 || Hq < 1 || Hkv < 1 || d_qk < 1 || d_v < 1) return B200ATTN_ERR_INVALID;
+  if (granularity != B200ATTN_SCALE_PER_HEAD && granularity != B200ATTN_SCALE_PER_BLOCK)
+    return B200ATTN_ERR_UNSUPPORTED;
+  if (hadamard != 0 && hadamard != 1) return B200ATTN_ERR_INVALID;
+  if (!(d_v == 128 && (d_qk == 128 || d_qk == 192))) return B200ATTN_ERR_UNSUPPORTED;
+  const void* ptrs[6] = {q, k, v, q_fp8, k_fp8, v_fp8};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return B200ATTN_ERR_INVALID;
+  const float* sptrs[3] = {q_scale, k_scale, v_scale};
+  for (const float* ptr : sptrs)
+    if (reinterpret_cast<uintptr_t>(ptr) & 3u) return B200ATTN_ERR_INVALID;
+  const int64_t nblk = (static_cast<int64_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  if (nblk > 0x7fffffff || static_cast<int64_t>(Hq) + 2 * static_cast<int64_t>(Hkv) > 65535 || B > 65535)
+    return B200ATTN_ERR_UNSUPPORTED;
+  const size_t need = b200attn_quantize_qkv_workspace_bytes(B, N, Hq, Hkv, granularity);
+  if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 3u)))
+    return B200ATTN_ERR_WORKSPACE;
+  int sm_count = 0;
+  const int dev_rc = device_ok(&sm_count);
+  if (dev_rc != B200ATTN_OK) return dev_rc;
+
+  b200::QkvQuant a;
+  a.x[0] = static_cast<const __nv_bfloat16*>(q);
+  a.x[1] = static_cast<const __nv_bfloat16*>(k);
+  a.x[2] = static_cast<const __nv_bfloat16*>(v);
+  a.y[0] = static_cast<uint8_t*>(q_fp8);
+  a.y[1] = static_cast<uint8_t*>(k_fp8);
+  a.y[2] = static_cast<uint8_t*>(v_fp8);
+  a.scale[0] = q_scale;
+  a.scale[1] = k_scale;
+  a.scale[2] = v_scale;
+  a.H[0] = Hq;
+  a.H[1] = Hkv;
+  a.H[2] = Hkv;
+  a.N = N;
+  a.nblk = static_cast<int>(nblk);
+  float* ws = static_cast<float*>(workspace);
+  a.partial[0] = ws;
+  a.partial[1] = ws ? ws + static_cast<size_t>(B) * Hq * nblk : nullptr;
+  a.partial[2] = ws ? ws + static_cast<size_t>(B) * (Hq + Hkv) * nblk : nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d_qk == 128)
+    return hadamard ? launch_quant_qkv<128, 128, true>(a, B, granularity, st)
+                    : launch_quant_qkv<128, 128, false>(a, B, granularity, st);
+  return hadamard ? launch_quant_qkv<192, 128, true>(a, B, granularity, st)
+                  : launch_quant_qkv<192, 128, false>(a, B, granularity, st);
+}
+
 
 // ---------------------------------------------------------------------------------------------
 // Per-head quantizer without any allocation: the partial-absmax scratch lives in

@@ -141,32 +141,26 @@ __device__ __forceinline__ float block_max(float m, float* red) {
   return m;
 }
 
-// Pass 1 of the per-head path: partial absmax of each 128-token block.
+// Pass 1 of the per-head path: partial absmax of 128-token block blk of (b, h).
 template <int D, bool HAD>
-__global__ void __launch_bounds__(kQuantThreads)
-    quant_absmax_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ partial, int N, int H) {
-  __shared__ float red[kQuantThreads / 32];
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+__device__ __forceinline__ void absmax_body(const __nv_bfloat16* __restrict__ x, float* __restrict__ partial, int N,
+                                            int H, int nblk, int blk, int h, int b, float* red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float v[QuantLayout<D>::ITERS][8];
   float m;
   load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, v, m);
   m = block_max(m, red);
-  if (threadIdx.x == 0) partial[(static_cast<size_t>(b) * H + h) * gridDim.x + blk] = m;
+  if (threadIdx.x == 0) partial[(static_cast<size_t>(b) * H + h) * nblk + blk] = m;
 }
 
 // Encode one 128-token block. PER_HEAD: amax is the max of the partials of
 // this head; otherwise the block's own.
 template <int D, bool HAD, bool PER_HEAD>
-__global__ void __launch_bounds__(kQuantThreads)
-    quant_encode_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
-                        float* __restrict__ scale, const float* __restrict__ partial, int N, int H) {
+__device__ __forceinline__ void encode_body(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
+                                            float* __restrict__ scale, const float* __restrict__ partial, int N,
+                                            int H, int nblk, int blk, int h, int b, float* red) {
   using L = QuantLayout<D>;
-  __shared__ float red[kQuantThreads / 32];
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nblk = gridDim.x;
-
   float v[L::ITERS][8];
   float m;
   load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, v, m);
@@ -203,6 +197,70 @@ __global__ void __launch_bounds__(kQuantThreads)
       }
     }
   }
+}
+
+template <int D, bool HAD>
+__global__ void __launch_bounds__(kQuantThreads)
+    quant_absmax_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ partial, int N, int H) {
+  __shared__ float red[kQuantThreads / 32];
+  absmax_body<D, HAD>(x, partial, N, H, gridDim.x, blockIdx.x, blockIdx.y, blockIdx.z, red);
+}
+
+template <int D, bool HAD, bool PER_HEAD>
+__global__ void __launch_bounds__(kQuantThreads)
+    quant_encode_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
+                        float* __restrict__ scale, const float* __restrict__ partial, int N, int H) {
+  __shared__ float red[kQuantThreads / 32];
+  encode_body<D, HAD, PER_HEAD>(x, y, scale, partial, N, H, gridDim.x, blockIdx.x, blockIdx.y, blockIdx.z, red);
+}
+
+// Q, K and V in one launch per pass: blockIdx.y walks the heads of Q, then K,
+// then V. The rotation (HAD) applies to Q and K only.
+struct QkvQuant {
+  const __nv_bfloat16* x[3];
+  uint8_t* y[3];
+  float* scale[3];
+  float* partial[3];
+  int H[3];
+  int N;
+  int nblk;
+};
+
+__device__ __forceinline__ int qkv_pick(const QkvQuant& a, int yidx, int& h) {
+  if (yidx < a.H[0]) {
+    h = yidx;
+    return 0;
+  }
+  if (yidx < a.H[0] + a.H[1]) {
+    h = yidx - a.H[0];
+    return 1;
+  }
+  h = yidx - a.H[0] - a.H[1];
+  return 2;
+}
+
+template <int DQK, int DV, bool HAD>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_kernel(const QkvQuant a) {
+  __shared__ float red[kQuantThreads / 32];
+  int h;
+  const int t = qkv_pick(a, blockIdx.y, h);
+  if (t < 2)
+    absmax_body<DQK, HAD>(a.x[t], a.partial[t], a.N, a.H[t], a.nblk, blockIdx.x, h, blockIdx.z, red);
+  else
+    absmax_body<DV, false>(a.x[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.x, h, blockIdx.z, red);
+}
+
+template <int DQK, int DV, bool HAD, bool PER_HEAD>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_kernel(const QkvQuant a) {
+  __shared__ float red[kQuantThreads / 32];
+  int h;
+  const int t = qkv_pick(a, blockIdx.y, h);
+  if (t < 2)
+    encode_body<DQK, HAD, PER_HEAD>(a.x[t], a.y[t], a.scale[t], a.partial[t], a.N, a.H[t], a.nblk, blockIdx.x, h,
+                                    blockIdx.z, red);
+  else
+    encode_body<DV, false, PER_HEAD>(a.x[2], a.y[2], a.scale[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.x, h,
+                                     blockIdx.z, red);
 }
 
 }  // namespace b200

@@ -149,6 +149,40 @@ int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale,
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * b200attn_quantize_qkv_workspace_bytes -- device workspace
+ * b200attn_quantize_qkv_fp8 needs: B*(Hq+2*Hkv)*ceil(N/128)*4 bytes for
+ * SCALE_PER_HEAD, 0 for SCALE_PER_BLOCK. Returns 0 for invalid sizes.
+ */
+size_t b200attn_quantize_qkv_workspace_bytes(int B, int N, int Hq, int Hkv, int granularity);
+
+/*
+ * b200attn_quantize_qkv_fp8 -- b200attn_quantize_fp8 applied to Q, K and V
+ * of one attention call, in one launch per pass (two for SCALE_PER_HEAD, one
+ * for SCALE_PER_BLOCK) instead of one or two per tensor. The rotation, when
+ * hadamard == 1, applies to Q and K; V is quantised unrotated. Codes and
+ * scales are bit-identical to three b200attn_quantize_fp8 calls (hadamard on
+ * the first two).
+ *
+ * q [B,N,Hq,d_qk], k [B,N,Hkv,d_qk], v [B,N,Hkv,d_v]: bf16 device pointers
+ * q_fp8, k_fp8, v_fp8: e4m3 outputs of the same shapes
+ * q_scale [B,Hq] or [B,Hq,ceil(N/128)], k_scale and v_scale [B,Hkv] or
+ *        [B,Hkv,ceil(N/128)]: fp32 outputs by granularity
+ * d_qk, d_v: (128, 128) or (192, 128)
+ * workspace: device scratch of b200attn_quantize_qkv_workspace_bytes bytes
+ *        (NULL allowed when that is 0); caller-owned, contents on entry do not
+ *        matter, concurrent calls need distinct workspaces
+ *
+ * Errors: INVALID, UNSUPPORTED (head dims, more than 65535 heads in total),
+ * WORKSPACE, CUDA.
+ */
+int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v,
+                              void* q_fp8, void* k_fp8, void* v_fp8,
+                              float* q_scale, float* k_scale, float* v_scale,
+                              int B, int N, int Hq, int Hkv, int d_qk, int d_v,
+                              int granularity, int hadamard,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * b200attn_quantize_fp8_static -- the per-head (B200ATTN_SCALE_PER_HEAD)
  * quantizer of b200attn_quantize_fp8, for callers that cannot allocate device
  * memory: code that runs inside a framework which owns the device heap (a

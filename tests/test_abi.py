@@ -116,3 +116,25 @@ def test_package_has_no_oracle_dependency():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", text, re.M), f
                 assert "attn_oracle" not in text and "liboracle" not in text, f
+
+
+def qkv(lib, ptr=FAKE, B=1, N=256, Hq=4, Hkv=2, dqk=128, dv=128, gran=0, had=0, ws=FAKE, wsb=1 << 20):
+    p = [ptr] * 9
+    return lib.b200attn_quantize_qkv_fp8(*p, B, N, Hq, Hkv, dqk, dv, gran, had, ws, wsb, None)
+
+
+def test_quantize_qkv_workspace_and_arguments_on_the_host(lib):
+    # one partial absmax per 128-token block of every Q, K and V head
+    assert lib.b200attn_quantize_qkv_workspace_bytes(2, 300, 4, 2, 0) == 2 * (4 + 2 * 2) * 3 * 4
+    assert lib.b200attn_quantize_qkv_workspace_bytes(2, 300, 4, 2, 1) == 0
+    assert lib.b200attn_quantize_qkv_workspace_bytes(0, 300, 4, 2, 0) == 0
+    assert qkv(lib, ptr=None) == -1
+    assert qkv(lib, ptr=FAKE + 4) == -1                     # misaligned
+    assert qkv(lib, N=0) == -1
+    assert qkv(lib, had=2) == -1
+    assert qkv(lib, dqk=64) == -2
+    assert qkv(lib, dv=192) == -2
+    assert qkv(lib, gran=3) == -2
+    assert qkv(lib, Hq=65535, Hkv=1) == -2                  # more heads than a grid dimension holds
+    assert qkv(lib, ws=None) == -5
+    assert qkv(lib, wsb=8) == -5

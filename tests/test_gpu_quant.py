@@ -52,3 +52,22 @@ def test_full_size_q_bit_exact(name, hadamard):
         ref_codes, ref_scale = oracle.quantize_fp8(f32(t), "head", rot)
         assert np.array_equal(scale, ref_scale)
         assert np.array_equal(codes, ref_codes)
+
+
+@pytest.mark.parametrize("shape", [(1, 300, 4, 2, 128), (2, 129, 2, 2, 192), (1, 1000, 8, 1, 128)])
+@pytest.mark.parametrize("granularity", ["head", "block"])
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_qkv_in_one_launch_bit_exact(shape, granularity, hadamard):
+    """Q, K and V quantised together: each tensor's codes and scales equal the
+    oracle's, with the rotation on Q and K only."""
+    B, N, Hq, Hkv, dqk = shape
+    g = torch.Generator().manual_seed(B * 7 + N + Hq + dqk)
+    q = (torch.randn(B, N, Hq, dqk, generator=g) * 3).to(torch.bfloat16)
+    k = (torch.randn(B, N, Hkv, dqk, generator=g) * torch.exp(torch.randn(Hkv, dqk, generator=g))).to(torch.bfloat16)
+    v = torch.randn(B, N, Hkv, 128, generator=g).to(torch.bfloat16)
+    outs = b2.quantize_qkv_fp8(q.cuda(), k.cuda(), v.cuda(), granularity=granularity, hadamard=hadamard)
+    assert b2.check() == 0
+    for t, rot, (c, s) in ((q, hadamard, outs[0:2]), (k, hadamard, outs[2:4]), (v, False, outs[4:6])):
+        ref_codes, ref_scale = oracle.quantize_fp8(f32(t), granularity, rot)
+        assert np.array_equal(s.cpu().numpy(), ref_scale)
+        assert np.array_equal(c.view(torch.uint8).cpu().numpy(), ref_codes)
