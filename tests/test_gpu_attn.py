@@ -12,7 +12,7 @@ import torch
 import oracle
 import workloads
 import bf16_causal_prefill_fwd_b200 as b2
-from helpers import (BF16_TOL, FP8_TOL, f32, gather_sample, oracle_fp8_inputs, oracle_on_sample,
+from helpers import (BF16_TOL, FP8_TOL, f32, gather_sample, oracle_fp8_inputs, oracle_on_sample, subset_problem,
                      sampled_rows, to_gpu_fp8)
 
 pytestmark = pytest.mark.gpu
@@ -321,3 +321,36 @@ def test_full_size_fp8_sampled(name, hadamard, monkeypatch):
         print(f"{name} fp8[{mode}] (hadamard={hadamard}) rel-rms {err:.2e}; "
               f"vs unquantised fp64 {oracle.rel_rms(got, ref):.2e}")
         assert err <= FP8_TOL
+
+
+# ---------------------------------------------------------------- sequence sweep, FP8 error at each N
+
+@pytest.mark.parametrize("N", [1024, 2048, 4096, 8192, 16384, 32768])
+def test_sweep_fp8_error_sampled(N):
+    """The Gaussian sweep (B = 32768/N) through the product path: Q, K, V
+    quantised on the GPU, FP8 attention. The oracle quantises the sampled heads
+    of batch 0 itself; their codes must equal the GPU's, and the output must
+    match fp64 attention on them (the error against the unquantised inputs is
+    printed, not gated)."""
+    w = workloads.sweep(N)
+    q, k, v = workloads.draw(w)
+    q8, sq, k8, sk, v8, sv = b2.quantize_qkv_fp8(q.cuda(), k.cuda(), v.cuda())
+    o = b2.attn_fwd(q8, k8, v8, q_scale=sq, k_scale=sk, v_scale=sv)
+    assert b2.check() == 0
+    heads = [0, w.Hq - 1]
+    rows = sampled_rows(N)
+    qs, ks, vs = (t[:1].contiguous() for t in subset_problem(q, k, v, heads))
+    codes, deq = oracle_fp8_inputs(qs, ks, vs)
+    G = w.Hq // w.Hkv
+    kvh = [h // G for h in heads]
+    gpu_codes = (q8.view(torch.uint8)[:1, :, heads], k8.view(torch.uint8)[:1, :, kvh],
+                 v8.view(torch.uint8)[:1, :, kvh])
+    for mine, ref in zip(gpu_codes, codes[0::2]):
+        assert np.array_equal(mine.cpu().numpy(), ref)
+    sub = list(range(len(heads)))
+    ref8, _ = oracle_on_sample(*deq, sub, rows)
+    ref, _ = oracle_on_sample(qs, ks, vs, sub, rows)
+    got = gather_sample(o, heads, rows)
+    err, err_unq = oracle.rel_rms(got, ref8), oracle.rel_rms(got, ref)
+    print(f"sweep N={N} B={w.B} fp8 rel-rms {err:.2e}; vs unquantised fp64 {err_unq:.2e}")
+    assert err <= FP8_TOL, err
