@@ -59,7 +59,12 @@
 // rescales; E shifts FP8 probabilities up so the e4m3 normal range covers more
 // binades. Both cancel exactly in O_acc / l.
 //
-// FP8 probabilities, two ways (a template switch, chosen on the host):
+// Probabilities on the FMA pipe (template switch FMA_P, chosen on the host):
+// for FP8 it selects Lean P below; for BF16 it sends one score in four through
+// a polynomial 2^x (exp2_fma_x2) instead of MUFU, which with one MUFU ex2 per
+// score is as busy as the tensor core.
+//
+// FP8 probabilities, two ways:
 //  * MUFU: P = e4m3(ex2(x)), round to nearest even.
 //  * Lean P ("ZYFA 如何工作？", Lean P：用一次乘加代替指数运算): read as an
 //    integer, the e4m3 code of 2^x is close to 8x + 56 (+8 per doubling), so the
@@ -105,7 +110,7 @@ struct AttnParams {
   float* lse;
 };
 
-template <int DQK, int DV, bool FP8, bool LEANP = false, bool SHARED_S = true>
+template <int DQK, int DV, bool FP8, bool FMA_P = false, bool SHARED_S = true>
 struct AttnCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int CHUNK_ELEMS = 128 / ESZ;  // elements in one 128-byte swizzled row
@@ -145,7 +150,6 @@ struct AttnCfg {
                                     1024 /*bars*/ + 1024 /*align*/;
   static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
   static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
-  static_assert(!LEANP || FP8, "Lean P builds e4m3 codes");
   static constexpr uint32_t IDESC_QK = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, kBN, false);
   static constexpr uint32_t IDESC_PV = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DVX, true);
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
@@ -185,6 +189,27 @@ __device__ __forceinline__ int unit_for(int k, int cta, int grid) {
   return (k & 1) ? base + (grid - 1 - cta) : base + cta;
 }
 
+// 2^x for two lanes on the FMA pipe, for the bf16 probabilities that do not go
+// through MUFU: Cody-Waite split x = j + f with j an integer and |f| <= 1/2
+// (adding and removing 1.5 * 2^23 rounds x to an integer), a degree-3
+// polynomial for 2^f (coefficients fitted to the relative error of 2^f on
+// [-1/2, 1/2]: at most 2.2e-4 in fp32, well below bf16's 2^-9), then j added to
+// the exponent field with an integer add. Inputs below -125 (masked keys among
+// them) give 0.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& r0, float& r1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float a0 = fmaxf(x0, -125.0f), a1 = fmaxf(x1, -125.0f);
+  float j0, j1, n0, n1, f0, f1, p0, p1;
+  ffma2_bcast(a0, a1, 1.0f, kRound, j0, j1);    // j + 1.5 * 2^23, j in the low mantissa bits
+  ffma2_bcast(j0, j1, 1.0f, -kRound, n0, n1);   // j
+  ffma2(n0, n1, -1.0f, -1.0f, a0, a1, f0, f1);  // f = a - j
+  ffma2_bcast(f0, f1, 0.05286737531423569f, 0.24215202033519745f, p0, p1);
+  ffma2(p0, p1, f0, f1, 0.6935867667198181f, 0.6935867667198181f, p0, p1);
+  ffma2(p0, p1, f0, f1, 0.9999627470970154f, 0.9999627470970154f, p0, p1);
+  r0 = x0 >= -125.0f ? __uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23)) : 0.0f;
+  r1 = x1 >= -125.0f ? __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23)) : 0.0f;
+}
+
 // Bounded mbarrier wait. Returns false if it gave up (2 s) or another role
 // already gave up; the first to give up records the timeout status.
 __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -208,11 +233,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort_flag);
 }
 
-template <int DQK, int DV, bool FP8, bool LEANP, bool SHARED_S>
+template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<DQK, DV, FP8, LEANP, SHARED_S>;
+  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S>;
   extern __shared__ uint8_t smem_raw[];
 
   // 1024-byte aligned base (128-byte swizzle atoms repeat every 1024 bytes).
@@ -637,8 +662,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             float x0, x1, x2, x3;
             ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), c_log2, nm, x0, x1);
             ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), c_log2, nm, x2, x3);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+            float p0, p1, p2, p3;
+            if (FMA_P && (c & 12) == 12) {  // one score in four off MUFU
+              exp2_fma_x2(x0, x1, p0, p1);
+              exp2_fma_x2(x2, x3, p2, p3);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+              p2 = ex2_approx(x2);
+              p3 = ex2_approx(x3);
+            }
             if ((c & 4) == 0) {
               fadd2(sa, sb, p0, p1);
               fadd2(sc, sd, p2, p3);
@@ -652,7 +685,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           l_blk = (sa + sb) + (sc + sd);
         } else if (mma_sum) {
           // codes only; the tensor core adds them up
-          if constexpr (LEANP) {
+          if constexpr (FMA_P) {
             const float A = c_blk * (8.0f / 126.0f);
             const float Bc = (8.0f * (C::E_SHIFT - m_run + lr) + 56.0f) * (1.0f / 126.0f);
 #pragma unroll
@@ -679,7 +712,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         } else {
           // acc: f16x2 partial sums of decode(code)/256 (8 adds per accumulator per block)
           uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          if constexpr (LEANP) {
+          if constexpr (FMA_P) {
             // w = (8 (c*S - m_run + E + lr) + 56) / 126, clamped below at 0; code = round(126 w)
             const float A = c_blk * (8.0f / 126.0f);
             const float Bc = (8.0f * (C::E_SHIFT - m_run + lr) + 56.0f) * (1.0f / 126.0f);

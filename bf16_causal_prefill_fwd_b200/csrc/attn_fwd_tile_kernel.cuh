@@ -42,7 +42,7 @@
 
 namespace b200 {
 
-template <int DQK, int DV, bool LEANP>
+template <int DQK, int DV, bool FMA_P>
 struct TileCfg {
   static constexpr int CHUNK_ELEMS = 128;        // e4m3 elements per 128-byte swizzled row
   static constexpr int CHUNK_BYTES = kBM * 128;  // 16 KiB
@@ -92,11 +92,11 @@ __device__ __forceinline__ TileUnit decode_tile_unit(int u, const AttnParams& p)
   return x;
 }
 
-template <int DQK, int DV, bool LEANP>
+template <int DQK, int DV, bool FMA_P>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = TileCfg<DQK, DV, LEANP>;
+  using C = TileCfg<DQK, DV, FMA_P>;
   extern __shared__ uint8_t smem_raw[];
 
   const uint32_t raw_u32 = smem_addr(smem_raw);
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(bMReady + 8 * b);
 
         // e4m3 codes in place (entry c/4 is already consumed)
-        if constexpr (LEANP) {
+        if constexpr (FMA_P) {
           const float A = c_log2 * (8.0f / 126.0f);
           const float Bc = (8.0f * (C::E_SHIFT - m_run) + 56.0f) * (1.0f / 126.0f);
 #pragma unroll

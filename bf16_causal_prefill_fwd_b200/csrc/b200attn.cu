@@ -65,6 +65,14 @@ bool fp8_lean_p() {
   return !(e && std::strcmp(e, "mufu") == 0);
 }
 
+// BF16 probabilities: every exponential on MUFU (default) or one in four by a
+// polynomial on the FMA pipe. B200ATTN_BF16_P=mixed selects the latter (read on
+// every call).
+bool bf16_fma_p() {
+  const char* e = std::getenv("B200ATTN_BF16_P");
+  return e && std::strcmp(e, "mixed") == 0;
+}
+
 int device_ok(int* sm_count) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return B200ATTN_ERR_CUDA;
@@ -77,15 +85,15 @@ int device_ok(int* sm_count) {
   return B200ATTN_OK;
 }
 
-template <int DQK, int DV, bool FP8, bool LEANP, bool SHARED_S>
+template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S>
 int launch_attn_t(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
-  using C = AttnCfg<DQK, DV, FP8, LEANP, SHARED_S>;
+  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, FP8, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, FP8, d_qk, p.Hkv, p.N, p.B) ||
       !make_tmap(&tv, v, FP8, d_v, p.Hkv, p.N, p.B))
     return B200ATTN_ERR_CUDA;
-  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, LEANP, SHARED_S>;
+  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, FMA_P, SHARED_S>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
@@ -102,23 +110,23 @@ bool shared_s() {
   return !(e && std::strcmp(e, "0") == 0);
 }
 
-template <int DQK, int DV, bool FP8, bool LEANP = false>
+template <int DQK, int DV, bool FP8, bool FMA_P = false>
 int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
-  if (shared_s()) return launch_attn_t<DQK, DV, FP8, LEANP, true>(q, k, v, p, d_qk, d_v, sm_count, stream);
-  return launch_attn_t<DQK, DV, FP8, LEANP, false>(q, k, v, p, d_qk, d_v, sm_count, stream);
+  if (shared_s()) return launch_attn_t<DQK, DV, FP8, FMA_P, true>(q, k, v, p, d_qk, d_v, sm_count, stream);
+  return launch_attn_t<DQK, DV, FP8, FMA_P, false>(q, k, v, p, d_qk, d_v, sm_count, stream);
 }
 
 // FP8 with per-head scales: one query tile per unit (attn_fwd_tile_kernel).
-template <int DQK, int DV, bool LEANP>
+template <int DQK, int DV, bool FMA_P>
 int launch_attn_tile(const void* q, const void* k, const void* v, AttnParams p, int d_qk, int d_v, int sm_count,
                      cudaStream_t stream) {
-  using C = b200::TileCfg<DQK, DV, LEANP>;
+  using C = b200::TileCfg<DQK, DV, FMA_P>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, true, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, true, d_qk, p.Hkv, p.N, p.B) ||
       !make_tmap(&tv, v, true, d_v, p.Hkv, p.N, p.B))
     return B200ATTN_ERR_CUDA;
-  auto kern = b200::attn_fwd_tile_kernel<DQK, DV, LEANP>;
+  auto kern = b200::attn_fwd_tile_kernel<DQK, DV, FMA_P>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
   p.n_units = p.B * p.Hq * p.n_kv;
@@ -215,6 +223,10 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   if (!fp8) {
+    if (bf16_fma_p()) {
+      if (d_qk == 128) return launch_attn<128, 128, false, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+      return launch_attn<192, 128, false, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+    }
     if (d_qk == 128) return launch_attn<128, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn<192, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
   }

@@ -418,6 +418,16 @@ __device__ __forceinline__ void ffma2_bcast(float a0, float a1, float b, float c
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
+// d = a * b + c elementwise on fp32 pairs.
+__device__ __forceinline__ void ffma2(float a0, float a1, float b0, float b1, float c0, float c1, float& d0,
+                                      float& d1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 // (s0, s1) += (a0, a1)
 __device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) {
   asm("{\n\t.reg .b64 ra, rs;\n\t"

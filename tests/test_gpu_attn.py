@@ -74,6 +74,22 @@ def fp8_kernel(request):
         os.environ["B200ATTN_FP8_TILE"] = old
 
 
+# BF16 forms every exponential on MUFU, or one in four by a polynomial on the
+# FMA pipe (B200ATTN_BF16_P=mixed); the tests marked with this fixture run both.
+BF16_P = ["mufu", "mixed"]
+
+
+@pytest.fixture
+def bf16_p(request):
+    old = os.environ.get("B200ATTN_BF16_P")
+    os.environ["B200ATTN_BF16_P"] = request.param
+    yield request.param
+    if old is None:
+        os.environ.pop("B200ATTN_BF16_P", None)
+    else:
+        os.environ["B200ATTN_BF16_P"] = old
+
+
 @pytest.fixture
 def fp8_p(request):
     old = os.environ.get("B200ATTN_FP8_P")
@@ -99,9 +115,10 @@ MUFU_LSE_ATOL = 0.061
 LEAN_LSE_ATOL = 0.121
 
 
+@pytest.mark.parametrize("bf16_p", BF16_P, indirect=True)
 @pytest.mark.parametrize("shape", SMALL)
 @pytest.mark.parametrize("causal", [True, False])
-def test_bf16_matches_oracle(shape, causal):
+def test_bf16_matches_oracle(shape, causal, bf16_p):
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq))
     o, lse = run_bf16(q, k, v, causal)
@@ -229,8 +246,9 @@ def test_causality_on_gpu():
 MANY_UNITS = (4, 32, 8, 1024, 128)
 
 
+@pytest.mark.parametrize("bf16_p", BF16_P, indirect=True)
 @pytest.mark.parametrize("causal", [True, False])
-def test_bf16_many_units_per_cta(causal):
+def test_bf16_many_units_per_cta(causal, bf16_p):
     B, Hq, Hkv, N, dqk = MANY_UNITS
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=21))
     o, _ = run_bf16(q, k, v, causal=causal)
@@ -256,13 +274,14 @@ def test_fp8_many_units_per_cta(causal, fp8_p, fp8_kernel):
     assert err <= FP8_TOL, err
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8-lean", "fp8-mufu", "fp8-lean-tile"])
+@pytest.mark.parametrize("dtype", ["bf16", "bf16-mixed", "fp8-lean", "fp8-mufu", "fp8-lean-tile"])
 def test_bitwise_deterministic_over_1000_launches(dtype, monkeypatch):
+    monkeypatch.setenv("B200ATTN_BF16_P", "mixed" if dtype == "bf16-mixed" else "mufu")
     if dtype.startswith("fp8"):
         monkeypatch.setenv("B200ATTN_FP8_P", dtype.split("-")[1])
         monkeypatch.setenv("B200ATTN_FP8_TILE", "1" if dtype.endswith("-tile") else "0")
     q, k, v = workloads.draw(workloads.gaussian(1, 8, 2, 2048, 128, 128, seed=8))
-    if dtype == "bf16":
+    if dtype.startswith("bf16"):
         args = (q.cuda(), k.cuda(), v.cuda())
         kw = {}
     else:
