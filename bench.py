@@ -114,6 +114,7 @@ class ClockSampler:
     def __init__(self, torch_device: int, interval_s: float = 0.01):
         self.samples = []
         self.window = []
+        self.energy_mj = []
         self.interval = interval_s
         self._stop = threading.Event()
         self.handle = None
@@ -151,6 +152,17 @@ class ClockSampler:
 
     def mark(self):
         self.window.append(time.perf_counter())
+        if self.handle is not None:
+            try:
+                self.energy_mj.append(self.nv.nvmlDeviceGetTotalEnergyConsumption(self.handle))
+            except Exception:  # noqa: BLE001 - counter not supported: no energy figure
+                pass
+
+    def energy_j(self):
+        """Joules between the first and last mark (NVML's total-energy counter), or None."""
+        if len(self.energy_mj) < 2:
+            return None
+        return (self.energy_mj[-1] - self.energy_mj[0]) / 1000.0
 
     def __exit__(self, *exc):
         self._stop.set()
@@ -336,8 +348,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         peak = bf16_peak * (2.0 if dtype == "fp8" else 1.0)
         fp8_p = os.environ.get("B200ATTN_FP8_P", "lean")
         kname = "attn_fwd_tile_kernel" if os.environ.get("B200ATTN_FP8_TILE") == "1" else "attn_fwd_kernel"
+        bf16_p = "mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed"
         kernel_key = (f"{kname}<{w.d_qk},{w.d_v},fp8,{'mufu' if fp8_p == 'mufu' else 'lean'}>"
-                      if dtype == "fp8" else f"attn_fwd_kernel<{w.d_qk},{w.d_v},bf16>")
+                      if dtype == "fp8" else f"attn_fwd_kernel<{w.d_qk},{w.d_v},bf16,{bf16_p}>")
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic_for(kernel_key, w.name),
                 "kernel": kernel_key, "kernel_ms": ams,
@@ -351,6 +364,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     with ClockSampler(local_rank) as clk:
         main = measure(args.dtype, clk)
     clocks = clk.summary()
+    # Energy of this GPU over the timed steps (NVML total-energy counter; the window also
+    # holds the L2-flush writes between steps, so TFLOP/J is slightly conservative).
+    joules = clk.energy_j()
+    energy = None
+    if joules and joules > 0:
+        energy = {"tflop_per_j": w.flops * args.steps / joules / 1e12, "joules": joules,
+                  "source": "NVML total energy consumption over the timed steps, this GPU, "
+                            "L2-flush writes between steps included"}
     other = None
     if not args.no_other_dtype:
         other_dtype = "bf16" if args.dtype == "fp8" else "fp8"
@@ -382,9 +403,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                        "l2": "256 MiB buffer written between timed steps (untimed); inputs exceed L2",
                        "settle": f"{args.settle_s} s of untimed back-to-back steps before timing",
                        "fp8_p": os.environ.get("B200ATTN_FP8_P", "lean") if args.dtype == "fp8" else None,
+                       "bf16_p": (("mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed")
+                                  if args.dtype == "bf16" else None),
                        "parallelism": f"replicas x{world}"},
             "roofline": main["roofline"],
             "clocks": clocks,
+            "energy": energy,
             "gpu_launches": main["launches"],
             "e2e": e2e,
             "cpu_baseline": cpu,

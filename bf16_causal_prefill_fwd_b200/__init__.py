@@ -8,6 +8,8 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     attn_func,
     attn_fwd,
+    attn_varlen_func,
+    attn_varlen_fwd,
     check,
     load_library,
     quantize_fp8,

@@ -53,6 +53,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.b200attn_quantize_qkv_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.b200attn_quantize_qkv_fp8.restype = i
     lib.b200attn_quantize_qkv_fp8.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp]
+    lib.b200attn_fwd_varlen_workspace_bytes.restype = sz
+    lib.b200attn_fwd_varlen_workspace_bytes.argtypes = [ctypes.POINTER(ctypes.c_int), i, i]
+    lib.b200attn_fwd_varlen.restype = i
+    lib.b200attn_fwd_varlen.argtypes = ([vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int)] + [i] * 8
+                                        + [vp, vp, vp, f, vp, vp, sz, vp])
     lib.b200attn_check.restype = i
     lib.b200attn_check.argtypes = [vp]
     lib.b200attn_strerror.restype = ctypes.c_char_p
@@ -130,6 +135,69 @@ def attn_fwd(q, k, v, *, causal: bool = True, softmax_scale: float | None = None
     if rc != 0:
         raise B200AttnError(rc, "b200attn_fwd")
     return (out, lse) if return_lse else out
+
+
+def _cu_array(cu_seqlens):
+    vals = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    return (ctypes.c_int * len(vals))(*vals), len(vals) - 1
+
+
+def attn_varlen_fwd(q, k, v, cu_seqlens, *, causal: bool = True, softmax_scale: float | None = None,
+                    q_scale=None, k_scale=None, v_scale=None, out=None, return_lse: bool = False,
+                    workspace=None, stream=None):
+    """Packed variable-length batch via b200attn_fwd_varlen: q [total,Hq,d_qk], k [total,Hkv,d_qk],
+    v [total,Hkv,d_v] (bf16, or e4m3 with per-head fp32 scales [Hq] / [Hkv]); sequence b owns rows
+    cu_seqlens[b]:cu_seqlens[b+1] (cu_seqlens: host ints, e.g. a list or a CPU tensor). Returns
+    bf16 [total,Hq,d_v] (and fp32 lse [Hq,total] if ``return_lse``)."""
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_cuda_contig(name, t)
+        if t.dim() != 3:
+            raise ValueError(f"{name} must be 3-D [total, H, d]")
+    fp8 = _is_fp8(q)
+    if fp8 != _is_fp8(k) or fp8 != _is_fp8(v) or (not fp8 and not (q.dtype == k.dtype == v.dtype == torch.bfloat16)):
+        raise ValueError("q, k, v must all be bf16 or all e4m3")
+    total, Hq, d_qk = q.shape
+    Hkv, d_v = k.shape[1], v.shape[2]
+    if k.shape != (total, Hkv, d_qk) or v.shape != (total, Hkv, d_v):
+        raise ValueError("shape mismatch between q, k and v")
+    cu, batch = _cu_array(cu_seqlens)
+    if out is None:
+        out = torch.empty((total, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device) if return_lse else None
+    if total == 0:  # nothing to compute (and no device memory to point at)
+        if batch < 1 or any(c != 0 for c in cu):
+            raise ValueError("cu_seqlens must be non-decreasing from 0 to total")
+        return (out, lse) if return_lse else out
+    if fp8:
+        for name, sc in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+            if sc is None:
+                raise ValueError(f"{name} is required for e4m3 inputs")
+            _check_cuda_contig(name, sc)
+    need = int(lib.b200attn_fwd_varlen_workspace_bytes(cu, batch, Hq))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.b200attn_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), cu, batch, total, Hq, Hkv, d_qk, d_v, 1 if causal else 0,
+        FP8_E4M3 if fp8 else BF16, _ptr(q_scale) if fp8 else None, _ptr(k_scale) if fp8 else None,
+        _ptr(v_scale) if fp8 else None, float(softmax_scale) if softmax_scale else 0.0, _ptr(lse), _ptr(workspace),
+        wbytes, _stream_handle(stream))
+    if rc != 0:
+        raise B200AttnError(rc, "b200attn_fwd_varlen")
+    return (out, lse) if return_lse else out
+
+
+def attn_varlen_func(q, k, v, cu_seqlens, softmax_scale: float | None = None, causal: bool = True, *,
+                     fp8: bool = False, hadamard: bool = False, return_lse: bool = False, stream=None):
+    """flash_attn_varlen_func-style call on packed bf16 [total, H, d] tensors (self-attention).
+    With ``fp8=True`` the packed Q, K, V are quantised to e4m3 with per-head scales first."""
+    if not fp8:
+        return attn_varlen_fwd(q, k, v, cu_seqlens, causal=causal, softmax_scale=softmax_scale,
+                               return_lse=return_lse, stream=stream)
+    q8, sq, k8, sk, v8, sv = quantize_qkv_fp8(q[None], k[None], v[None], hadamard=hadamard, stream=stream)
+    return attn_varlen_fwd(q8[0], k8[0], v8[0], cu_seqlens, causal=causal, softmax_scale=softmax_scale,
+                           q_scale=sq[0], k_scale=sk[0], v_scale=sv[0], return_lse=return_lse, stream=stream)
 
 
 def quantize_workspace_bytes(B, N, H, d, granularity="head") -> int:

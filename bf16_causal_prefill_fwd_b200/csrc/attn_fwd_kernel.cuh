@@ -95,6 +95,12 @@ constexpr int kStatusTimeout = -4;                 // B200ATTN_ERR_TIMEOUT
 
 __device__ int g_b200attn_status;  // device status word, read and cleared by b200attn_check
 
+// A unit of packed variable-length work: the sequence's first token row in the
+// packed tensors, its length, the query head and the pair index.
+struct VarlenUnit {
+  int row0, len, hq, pair;
+};
+
 struct AttnParams {
   int B, Hq, Hkv, N, G;
   int n_kv;      // ceil(N / 128): key blocks = query tiles
@@ -108,6 +114,10 @@ struct AttnParams {
   const float* v_scale;
   __nv_bfloat16* o;
   float* lse;
+  // Variable-length batches (NULL for [B, N, H, d] batches): sequences are packed
+  // along the token dimension (B = 1, N = total tokens) and units are read from
+  // this table, already ordered longest first.
+  const VarlenUnit* units;
 };
 
 template <int DQK, int DV, bool FP8, bool FMA_P = false, bool SHARED_S = true>
@@ -161,10 +171,27 @@ struct AttnCfg {
 
 struct Unit {
   int b, hq, hkv, pair, n0, n1;
+  int row0;  // first token row of the sequence (0 for [B, N, H, d] batches)
+  int len;   // sequence length
 };
 
 __device__ __forceinline__ Unit decode_unit(int u, const AttnParams& p) {
   Unit x;
+  if (p.units != nullptr) {
+    const VarlenUnit v = p.units[u];
+    const int n_kv = (v.len + kBN - 1) / kBN;
+    x.b = 0;
+    x.hq = v.hq;
+    x.hkv = v.hq / p.G;
+    x.pair = v.pair;
+    x.row0 = v.row0;
+    x.len = v.len;
+    x.n0 = p.causal ? min(2 * x.pair + 1, n_kv) : n_kv;
+    x.n1 = p.causal ? min(2 * x.pair + 2, n_kv) : n_kv;
+    return x;
+  }
+  x.row0 = 0;
+  x.len = p.N;
   const int bh = p.B * p.Hq;
   const int rnd = u / bh;
   const int r = u - rnd * bh;
@@ -353,7 +380,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int c = 0; c < C::QK_CHUNKS; ++c)
               tma_load_4d_hint(sQ + t * C::Q_BYTES + c * C::CHUNK_BYTES, &tmQ, bar, c * C::CHUNK_ELEMS, x.hq,
-                               (2 * x.pair + t) * kBM, x.b, pol_q);
+                               x.row0 + (2 * x.pair + t) * kBM, x.b, pol_q);
           }
         }
         for (int j = 0; j < x.n1 && ok; ++j, ++it) {
@@ -363,8 +390,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t bar = bFull + 8 * s;
           mbar_arrive_expect_tx(bar, slot_bytes);
           for (int c = 0; c < chunks; ++c)
-            tma_load_4d_hint(ring + s * slot_bytes + c * C::CHUNK_BYTES, tm, bar, c * C::CHUNK_ELEMS, x.hkv, j * kBN,
-                             x.b, pol_kv);
+            tma_load_4d_hint(ring + s * slot_bytes + c * C::CHUNK_BYTES, tm, bar, c * C::CHUNK_ELEMS, x.hkv,
+                             x.row0 + j * kBN, x.b, pol_kv);
         }
         first = false;
       }
@@ -606,8 +633,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int c = 0; c < 128; ++c)
               if (c > lim) sr[c] = __float_as_uint(-INFINITY);
           }
-        } else if (kv0 + kBN > p.N) {
-          const int lim = p.N - kv0;
+        } else if (kv0 + kBN > x.len) {
+          const int lim = x.len - kv0;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
@@ -828,8 +855,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l_run = __uint_as_float(lr16[0]);
       }
       const float inv_l = v_mult / l_run;
-      const bool row_ok = qrow < p.N;
-      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(x.b) * p.N + (row_ok ? qrow : 0)) * p.Hq + x.hq) * DV;
+      const bool row_ok = qrow < x.len;  // rows past the sequence belong to the next one (or to no one)
+      __nv_bfloat16* orow =
+          p.o + ((static_cast<size_t>(x.b) * p.N + x.row0 + (row_ok ? qrow : 0)) * p.Hq + x.hq) * DV;
 #pragma unroll 1
       for (int cc = 0; cc < DV; cc += 32) {
         uint32_t orr[32];
@@ -847,7 +875,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       if (p.lse != nullptr && row_ok)
-        p.lse[(static_cast<size_t>(x.b) * p.Hq + x.hq) * p.N + qrow] =
+        p.lse[(static_cast<size_t>(x.b) * p.Hq + x.hq) * p.N + x.row0 + qrow] =
             (m_run + __log2f(l_run) - C::E_SHIFT) * 0.6931471805599453f;
       tc_fence_before();
       mbar_arrive(bOe);

@@ -104,6 +104,46 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o,
                  float* lse, void* stream);
 
 /*
+ * b200attn_fwd_varlen_workspace_bytes -- device workspace b200attn_fwd_varlen
+ * needs for this batch: 16 bytes per work unit, one unit per (sequence, query
+ * head, pair of 128-row query tiles). cu_seqlens is the HOST array of
+ * b200attn_fwd_varlen. Returns 0 for invalid arguments (and for a batch of
+ * empty sequences).
+ */
+size_t b200attn_fwd_varlen_workspace_bytes(const int* cu_seqlens, int batch, int Hq);
+
+/*
+ * b200attn_fwd_varlen -- b200attn_fwd on a batch of sequences of different
+ * lengths packed along the token dimension, as flash_attn_varlen_func takes
+ * them (self-attention: the same lengths for queries and keys).
+ *
+ * q [total, Hq, d_qk], k [total, Hkv, d_qk], v [total, Hkv, d_v], o [total, Hq,
+ *        d_v]: device pointers, contiguous; sequence b owns token rows
+ *        [cu_seqlens[b], cu_seqlens[b+1])
+ * cu_seqlens  HOST int array [batch + 1]: 0 = cu[0] <= cu[1] <= ... <=
+ *        cu[batch] = total; empty sequences are allowed
+ * q_scale, k_scale, v_scale  FP8 only: per-head scales over the packed
+ *        tensors, [Hq] and [Hkv] (b200attn_quantize_fp8 with B = 1, N = total);
+ *        per-block scales are not supported here
+ * lse    optional fp32 [Hq, total]
+ * workspace  device memory of b200attn_fwd_varlen_workspace_bytes bytes,
+ *        16-byte aligned, caller-owned; the call writes the unit table there
+ *        (a host-to-device copy on `stream`) and the kernel reads it, so it
+ *        must stay untouched until the kernel has finished
+ * Other arguments as in b200attn_fwd. Each sequence is computed exactly as
+ * b200attn_fwd computes one batch entry.
+ *
+ * Errors: INVALID (as b200attn_fwd, and for a cu_seqlens array that is not
+ * non-decreasing from 0 to total), UNSUPPORTED, WORKSPACE, CUDA.
+ */
+int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                        const int* cu_seqlens, int batch, int total,
+                        int Hq, int Hkv, int d_qk, int d_v, int causal, int dtype,
+                        const float* q_scale, const float* k_scale, const float* v_scale,
+                        float softmax_scale, float* lse,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * b200attn_quantize_workspace_bytes -- device workspace b200attn_quantize_fp8
  * needs for these sizes: B*H*ceil(N/128)*4 bytes for SCALE_PER_HEAD (one
  * partial absmax per 128-token block), 0 for SCALE_PER_BLOCK. Returns 0 for

@@ -138,3 +138,21 @@ def test_quantize_qkv_workspace_and_arguments_on_the_host(lib):
     assert qkv(lib, Hq=65535, Hkv=1) == -2                  # more heads than a grid dimension holds
     assert qkv(lib, ws=None) == -5
     assert qkv(lib, wsb=8) == -5
+
+
+def test_varlen_workspace_and_arguments_on_the_host(lib):
+    IntArr = ctypes.c_int * 4
+    cu = IntArr(0, 100, 100, 400)      # 1 + 0 + 2 pairs of 128-row tiles
+    assert lib.b200attn_fwd_varlen_workspace_bytes(cu, 3, 4) == (1 + 0 + 2) * 4 * 16
+
+    def call(cu_vals, total, ws=FAKE, wsb=1 << 20, dtype=0, q=FAKE):
+        arr = (ctypes.c_int * len(cu_vals))(*cu_vals)
+        return lib.b200attn_fwd_varlen(q, FAKE, FAKE, FAKE, arr, len(cu_vals) - 1, total, 4, 2, 128, 128, 1,
+                                       dtype, None, None, None, 0.0, None, ws, wsb, None)
+    assert call([0, 100, 50, 400], 400) == -1        # decreasing
+    assert call([1, 100, 400], 400) == -1            # not starting at 0
+    assert call([0, 100, 399], 400) == -1            # not ending at total
+    assert call([0, 100, 400], 400, q=None) == -1
+    assert call([0, 100, 400], 400, dtype=1) == -1   # FP8 without scales
+    assert call([0, 100, 400], 400, ws=None) == -5
+    assert call([0, 100, 400], 400, wsb=16) == -5

@@ -74,8 +74,9 @@ def fp8_kernel(request):
         os.environ["B200ATTN_FP8_TILE"] = old
 
 
-# BF16 forms every exponential on MUFU, or one in four by a polynomial on the
-# FMA pipe (B200ATTN_BF16_P=mixed); the tests marked with this fixture run both.
+# BF16 forms one exponential in four by a polynomial on the FMA pipe (default)
+# or all of them on MUFU (B200ATTN_BF16_P=mufu); the tests marked with this
+# fixture run both.
 BF16_P = ["mufu", "mixed"]
 
 
