@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--workload", default="gqa7b")
     ap.add_argument("--n", type=int, default=None, help="sequence length override")
     ap.add_argument("--hadamard", action="store_true", help="rotate Q and K before FP8 quantisation")
+    ap.add_argument("--energy-s", type=float, default=2.0,
+                    help="seconds of back-to-back steps for the TFLOP/J figure (0: skip)")
     ap.add_argument("--fp8-p", choices=["lean", "mufu"], default=None,
                     help="how the FP8 kernel forms probabilities (default: the library default, Lean P)")
     ap.add_argument("--settle-s", type=float, default=1.0,
@@ -114,7 +116,6 @@ class ClockSampler:
     def __init__(self, torch_device: int, interval_s: float = 0.01):
         self.samples = []
         self.window = []
-        self.energy_mj = []
         self.interval = interval_s
         self._stop = threading.Event()
         self.handle = None
@@ -152,17 +153,6 @@ class ClockSampler:
 
     def mark(self):
         self.window.append(time.perf_counter())
-        if self.handle is not None:
-            try:
-                self.energy_mj.append(self.nv.nvmlDeviceGetTotalEnergyConsumption(self.handle))
-            except Exception:  # noqa: BLE001 - counter not supported: no energy figure
-                pass
-
-    def energy_j(self):
-        """Joules between the first and last mark (NVML's total-energy counter), or None."""
-        if len(self.energy_mj) < 2:
-            return None
-        return (self.energy_mj[-1] - self.energy_mj[0]) / 1000.0
 
     def __exit__(self, *exc):
         self._stop.set()
@@ -315,6 +305,34 @@ def time_path(path: Path, steps: int, warmup: int, settle_s: float, flush, dist_
     return step_ms, attn_ms
 
 
+def measure_energy(clk, path, flops_per_step: float, seconds: float):
+    """TFLOP/J of this GPU: steps run back to back for `seconds`, energy from NVML's
+    total-energy counter (mJ) read before and after. A separate, longer window than
+    the timed steps, because the counter advances in coarse increments."""
+    if seconds <= 0 or clk.handle is None:
+        return None
+    nv, h = clk.nv, clk.handle
+    try:
+        torch.cuda.synchronize()
+        e0, t0, n = nv.nvmlDeviceGetTotalEnergyConsumption(h), time.perf_counter(), 0
+        while True:
+            for _ in range(10):
+                path.step()
+            n += 10
+            torch.cuda.synchronize()
+            if time.perf_counter() - t0 >= seconds:
+                break
+        e1, t1 = nv.nvmlDeviceGetTotalEnergyConsumption(h), time.perf_counter()
+    except Exception:  # noqa: BLE001 - counter not supported on this GPU
+        return None
+    joules = (e1 - e0) / 1000.0
+    if joules <= 0:
+        return None
+    return {"tflop_per_j": flops_per_step * n / joules / 1e12, "joules": joules, "watts": joules / (t1 - t0),
+            "steps": n, "seconds": t1 - t0,
+            "source": "NVML total energy consumption of this GPU over steps run back to back (no L2 flush)"}
+
+
 def max_over_ranks(x: float, dist_on: bool, device: str = "cuda") -> float:
     """The slowest rank's value: every rank contributes its own timing, all get the max."""
     if not dist_on:
@@ -364,14 +382,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     with ClockSampler(local_rank) as clk:
         main = measure(args.dtype, clk)
     clocks = clk.summary()
-    # Energy of this GPU over the timed steps (NVML total-energy counter; the window also
-    # holds the L2-flush writes between steps, so TFLOP/J is slightly conservative).
-    joules = clk.energy_j()
-    energy = None
-    if joules and joules > 0:
-        energy = {"tflop_per_j": w.flops * args.steps / joules / 1e12, "joules": joules,
-                  "source": "NVML total energy consumption over the timed steps, this GPU, "
-                            "L2-flush writes between steps included"}
+    energy = measure_energy(clk, Path(b2, q, k, v, args.dtype, args.hadamard), w.flops, args.energy_s)
     other = None
     if not args.no_other_dtype:
         other_dtype = "bf16" if args.dtype == "fp8" else "fp8"
