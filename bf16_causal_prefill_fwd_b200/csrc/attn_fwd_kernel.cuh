@@ -128,10 +128,6 @@ struct AttnCfg {
   static constexpr int QK_CHUNKS = (DQK + CHUNK_ELEMS - 1) / CHUNK_ELEMS;
   static constexpr int V_CHUNKS = (DV + CHUNK_ELEMS - 1) / CHUNK_ELEMS;
   static constexpr int Q_BYTES = QK_CHUNKS * CHUNK_BYTES;
-  // Q buffers per tile: with two, the next unit's Q tiles load while this unit
-  // runs (units are short for short sequences). Only e4m3 at d_qk = 128 leaves
-  // shared memory for it next to K and V rings of four or more slots.
-  static constexpr int QB = (FP8 && DQK == 128) ? 2 : 1;
   static constexpr int K_BYTES = QK_CHUNKS * CHUNK_BYTES;
   static constexpr int V_BYTES = V_CHUNKS * CHUNK_BYTES;
   static constexpr int STAGE_BYTES = K_BYTES > V_BYTES ? K_BYTES : V_BYTES;
@@ -154,13 +150,13 @@ struct AttnCfg {
   static constexpr int ONES_BYTES = RS ? CHUNK_BYTES : 0;
   // Separate K and V rings, sized from what shared memory has left.
   static constexpr int SMEM_AVAIL = 227 * 1024 - 2048;  // minus barriers and alignment slack
-  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * QB * Q_BYTES - ONES_BYTES;
+  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BYTES - ONES_BYTES;
   static constexpr int RING_PAIRS = RING_AVAIL / (K_BYTES + V_BYTES);
   static constexpr int SV = RING_PAIRS >= 2 ? (RING_PAIRS > 4 ? 4 : RING_PAIRS) : 1;
   static constexpr int SK_FIT = (RING_AVAIL - SV * V_BYTES) / K_BYTES;
   static constexpr int SK = SK_FIT > 6 ? 6 : SK_FIT;
-  static constexpr int NUM_BARS = 4 + 4 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
-  static constexpr int SMEM_BYTES = 2 * QB * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES +
+  static constexpr int NUM_BARS = 2 + 2 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
+  static constexpr int SMEM_BYTES = 2 * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES +
                                     1024 /*bars*/ + 1024 /*align*/;
   static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
   static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
@@ -277,7 +273,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
 
   const uint32_t sQ = base_u32;                              // 2 query tiles
-  const uint32_t sK = sQ + 2 * C::QB * C::Q_BYTES;          // K ring (Q: [tile][QB])
+  const uint32_t sK = sQ + 2 * C::Q_BYTES;                   // K ring
   const uint32_t sV = sK + C::SK * C::K_BYTES;               // V ring
   const uint32_t sOnes = sV + C::SV * C::V_BYTES;          // RS: e4m3 ones, B columns d_v..d_v+15
   const uint32_t sBar = sOnes + C::ONES_BYTES;
@@ -286,9 +282,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NUM_BARS + 4);
 
   // barrier addresses
-  const uint32_t bQFull = sBar;                          // [2][2] TMA -> QK issuer, per tile and Q buffer
-  const uint32_t bQEmpty = bQFull + 32;                  // [2][2] QK issuer -> TMA
-  const uint32_t bKFull = bQEmpty + 32;                  // [SK] TMA -> QK issuer
+  const uint32_t bQFull = sBar;                          // [2]  TMA -> QK issuer
+  const uint32_t bQEmpty = bQFull + 16;                  // [2]  QK issuer -> TMA
+  const uint32_t bKFull = bQEmpty + 16;                  // [SK] TMA -> QK issuer
   const uint32_t bKEmpty = bKFull + 8 * C::SK;           // [SK] QK issuer -> TMA
   const uint32_t bVFull = bKEmpty + 8 * C::SK;           // [SV] TMA -> PV issuer
   const uint32_t bVEmpty = bVFull + 8 * C::SV;           // [SV] PV issuer -> TMA
@@ -310,10 +306,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       for (int t = 0; t < 2; ++t) {
-        for (int qb = 0; qb < 2; ++qb) {
-          mbar_init(bQFull + 8 * (2 * t + qb), 1);
-          mbar_init(bQEmpty + 8 * (2 * t + qb), 1);
-        }
+        mbar_init(bQFull + 8 * t, 1);
+        mbar_init(bQEmpty + 8 * t, 1);
         mbar_init(bSFull + 8 * t, 1);
         if (t == 0) mbar_init(bSFree, 128);
         for (int b = 0; b < C::PBX; ++b) {
@@ -368,23 +362,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const CUtensorMap* tm = is_k ? &tmK : &tmV;
       const int chunks = is_k ? C::QK_CHUNKS : C::V_CHUNKS;
       uint32_t it = 0;
-      bool ok = true;
+      uint32_t qe_par[2] = {0, 0};
+      bool first = true, ok = true;
       for (int k = 0; ok; ++k) {
         const int u = unit_for(k, blockIdx.x, gridDim.x);
         if (u >= p.n_units) break;
         const Unit x = decode_unit(u, p);
         if (is_k) {
-          // Q tiles of unit k into buffer k % QB, once unit k-QB's last QK^T has read it
-          const int qb = k % C::QB;
           for (int t = 0; t < 2 && ok; ++t) {
-            if (k >= C::QB && !(ok = mbar_wait(bQEmpty + 8 * (2 * t + qb), ((k / C::QB) - 1) & 1, abort_flag)))
-              break;
-            const uint32_t bar = bQFull + 8 * (2 * t + qb);
+            if (!first) {
+              ok = mbar_wait(bQEmpty + 8 * t, qe_par[t], abort_flag);
+              qe_par[t] ^= 1;
+              if (!ok) break;
+            }
+            const uint32_t bar = bQFull + 8 * t;
             mbar_arrive_expect_tx(bar, C::Q_BYTES);
 #pragma unroll
             for (int c = 0; c < C::QK_CHUNKS; ++c)
-              tma_load_4d_hint(sQ + (t * C::QB + qb) * C::Q_BYTES + c * C::CHUNK_BYTES, &tmQ, bar,
-                               c * C::CHUNK_ELEMS, x.hq, x.row0 + (2 * x.pair + t) * kBM, x.b, pol_q);
+              tma_load_4d_hint(sQ + t * C::Q_BYTES + c * C::CHUNK_BYTES, &tmQ, bar, c * C::CHUNK_ELEMS, x.hq,
+                               x.row0 + (2 * x.pair + t) * kBM, x.b, pol_q);
           }
         }
         for (int j = 0; j < x.n1 && ok; ++j, ++it) {
@@ -397,6 +393,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_load_4d_hint(ring + s * slot_bytes + c * C::CHUNK_BYTES, tm, bar, c * C::CHUNK_ELEMS, x.hkv,
                              x.row0 + j * kBN, x.b, pol_kv);
         }
+        first = false;
       }
       if (!ok) __nanosleep(200000);  // let copies already in flight land before the CTA exits
     }
@@ -410,12 +407,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t k_lo0 = sdesc_lo(sK, 16);
       const uint32_t v_lo0 = sdesc_lo(sV, C::CHUNK_BYTES);
       uint32_t gb[2] = {0, 0};  // key blocks tile t has processed in earlier units
-      int qb = 0;               // Q buffer of the current unit
+      uint32_t q_par = 0;
       uint32_t oe_par[2] = {0, 0};
       bool first = true, ok = true;
       // QK^T for tile t into S_t from K slot s.
       auto issue_qk = [&](int t, uint32_t s) {
-        const uint32_t a_lo = q_lo0 + (t * C::QB + qb) * (C::Q_BYTES >> 4);
+        const uint32_t a_lo = q_lo0 + t * (C::Q_BYTES >> 4);
         const uint32_t b_lo = k_lo0 + s * (C::K_BYTES >> 4);
 #pragma unroll
         for (int kk = 0; kk < DQK / C::MMA_K; ++kk) {
@@ -455,10 +452,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // previous S out. Warp 2: O_t += P_t(j) V_j once the softmax has written
           // P_t(j) (and rescaled O_t).
           if (warp == 1) {
-            qb = k % C::QB;
-            const uint32_t qpar = (k / C::QB) & 1;
-            ok = mbar_wait(bQFull + 8 * qb, qpar, abort_flag) && mbar_wait(bQFull + 8 * (2 + qb), qpar, abort_flag);
+            ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
             if (!ok) break;
+            q_par ^= 1;
             for (int j = 0; j < x.n1 && ok; ++j) {
               uint32_t s;
               if (!(ok = take(bKFull, C::SK, kit, s))) break;
@@ -470,7 +466,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tc_fence_after();
                 issue_qk(t, s);
                 tc_commit(bSFull + 8 * t);
-                if (j == n_t - 1) tc_commit(bQEmpty + 8 * (2 * t + qb));
+                if (j == n_t - 1) tc_commit(bQEmpty + 8 * t);
               }
               if (!ok) break;
               tc_commit(bKEmpty + 8 * s);
@@ -505,17 +501,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // order, so PV_t(j-1) has read P (in S_t's columns) before S_t(j)
           // overwrites them, and each tile's PV and next QK^T run back to back.
           if (warp != 1) break;
-          qb = k % C::QB;
-          const uint32_t qpar = (k / C::QB) & 1;
-          ok = mbar_wait(bQFull + 8 * qb, qpar, abort_flag) && mbar_wait(bQFull + 8 * (2 + qb), qpar, abort_flag);
+          ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
           if (!ok) break;
+          q_par ^= 1;
           uint32_t ks;
           if (!(ok = take(bKFull, C::SK, kit, ks))) break;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
             issue_qk(t, ks);
             tc_commit(bSFull + 8 * t);
-            if ((t ? x.n1 : x.n0) == 1) tc_commit(bQEmpty + 8 * (2 * t + qb));
+            if ((t ? x.n1 : x.n0) == 1) tc_commit(bQEmpty + 8 * t);
           }
           tc_commit(bKEmpty + 8 * ks);
           for (int i = 1; i <= x.n1 && ok; ++i) {
@@ -542,7 +537,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               if (i < n_t) {
                 issue_qk(t, ks);
                 tc_commit(bSFull + 8 * t);
-                if (i == n_t - 1) tc_commit(bQEmpty + 8 * (2 * t + qb));
+                if (i == n_t - 1) tc_commit(bQEmpty + 8 * t);
               }
             }
             if (!ok) break;
