@@ -178,15 +178,19 @@ class ClockSampler:
 # reference arm / CPU baseline: the fp64 oracle on a bounded sample of the same workload
 # ---------------------------------------------------------------------------------------------
 
+def workload_desc(w: workloads.Workload) -> str:
+    """The workload named by its sizes; both arms print the same string."""
+    return (f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d_qk={w.d_qk} d_v={w.d_v} causal, "
+            f"seed {w.seed}")
+
+
 def oracle_sample(q, k, v, w: workloads.Workload, target_s: float, max_rows: int | None = None):
     """Time the fp64 oracle on rows of query head 0 (batch 0), rows spread over the sequence,
     growing the sample until it has taken about target_s. Returns (TFLOP/s, desc, seconds)."""
     import oracle
-    G = w.Hq // w.Hkv
     qs = q[0:1, :, 0:1].float().numpy().astype(np.float64)
     ks = k[0:1, :, 0:1].float().numpy().astype(np.float64)
     vs = v[0:1, :, 0:1].float().numpy().astype(np.float64)
-    _ = G
     rng = np.random.default_rng(0)
     n_rows, flops, secs = 64, 0.0, 0.0
     done_rows = 0
@@ -223,7 +227,7 @@ def run_reference(args, rank: int, world: int):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.flops / (val * 1e12) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name} B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d_qk={w.d_qk} d_v={w.d_v} causal",
+        "config": {"workload": workload_desc(w),
                    "sample": desc,
                    "ms_per_step": "the whole workload's FLOPs at the sampled rate (each timed step is a sample)"},
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
@@ -405,8 +409,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8_e4m3" if args.dtype == "fp8" else "bf16", "data": "synthetic",
-            "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d_qk={w.d_qk} "
-                                   f"d_v={w.d_v} causal, seed {w.seed}",
+            "config": {"workload": workload_desc(w),
                        "step": ("e4m3 quantizer on Q,K,V (per-head scales"
                                 + (", Hadamard on Q,K" if args.hadamard else "") + ") + FP8 attention")
                        if args.dtype == "fp8" else "BF16 attention",
