@@ -165,7 +165,7 @@ int launch_quant(const void* x, void* y, float* scale, int B, int N, int H, int 
 
 template <int DQK, int DV, bool HAD>
 int launch_quant_qkv(const b200::QkvQuant& a, int B, int gran, cudaStream_t stream) {
-  const dim3 grid(a.nblk, a.H[0] + a.H[1] + a.H[2], B);
+  const dim3 grid(a.H[0] + a.H[1] + a.H[2], a.nblk, B);
   if (gran == B200ATTN_SCALE_PER_HEAD) {
     b200::quant_qkv_absmax_kernel<DQK, DV, HAD><<<grid, b200::kQuantThreads, 0, stream>>>(a);
     b200::quant_qkv_encode_kernel<DQK, DV, HAD, true><<<grid, b200::kQuantThreads, 0, stream>>>(a);
@@ -417,7 +417,7 @@ int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v, void*
   for (const float* ptr : sptrs)
     if (reinterpret_cast<uintptr_t>(ptr) & 3u) return B200ATTN_ERR_INVALID;
   const int64_t nblk = (static_cast<int64_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
-  if (nblk > 0x7fffffff || static_cast<int64_t>(Hq) + 2 * static_cast<int64_t>(Hkv) > 65535 || B > 65535)
+  if (nblk > 65535 || static_cast<int64_t>(Hq) + 2 * static_cast<int64_t>(Hkv) > 0x7fffffff || B > 65535)
     return B200ATTN_ERR_UNSUPPORTED;
   const size_t need = b200attn_quantize_qkv_workspace_bytes(B, N, Hq, Hkv, granularity);
   if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 3u)))

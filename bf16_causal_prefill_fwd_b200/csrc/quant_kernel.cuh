@@ -214,8 +214,11 @@ __global__ void __launch_bounds__(kQuantThreads)
   encode_body<D, HAD, PER_HEAD>(x, y, scale, partial, N, H, gridDim.x, blockIdx.x, blockIdx.y, blockIdx.z, red);
 }
 
-// Q, K and V in one launch per pass: blockIdx.y walks the heads of Q, then K,
-// then V. The rotation (HAD) applies to Q and K only.
+// Q, K and V in one launch per pass: blockIdx.x walks the heads of Q, then K,
+// then V, and blockIdx.y the 128-token blocks. With the heads fastest, CTAs
+// that run at the same time read whole token rows ([H, d] is contiguous in
+// memory) instead of one head's 256-byte slice of many rows. The rotation
+// (HAD) applies to Q and K only.
 struct QkvQuant {
   const __nv_bfloat16* x[3];
   uint8_t* y[3];
@@ -226,16 +229,16 @@ struct QkvQuant {
   int nblk;
 };
 
-__device__ __forceinline__ int qkv_pick(const QkvQuant& a, int yidx, int& h) {
-  if (yidx < a.H[0]) {
-    h = yidx;
+__device__ __forceinline__ int qkv_pick(const QkvQuant& a, int hidx, int& h) {
+  if (hidx < a.H[0]) {
+    h = hidx;
     return 0;
   }
-  if (yidx < a.H[0] + a.H[1]) {
-    h = yidx - a.H[0];
+  if (hidx < a.H[0] + a.H[1]) {
+    h = hidx - a.H[0];
     return 1;
   }
-  h = yidx - a.H[0] - a.H[1];
+  h = hidx - a.H[0] - a.H[1];
   return 2;
 }
 
@@ -243,23 +246,23 @@ template <int DQK, int DV, bool HAD>
 __global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_kernel(const QkvQuant a) {
   __shared__ float red[kQuantThreads / 32];
   int h;
-  const int t = qkv_pick(a, blockIdx.y, h);
+  const int t = qkv_pick(a, blockIdx.x, h);
   if (t < 2)
-    absmax_body<DQK, HAD>(a.x[t], a.partial[t], a.N, a.H[t], a.nblk, blockIdx.x, h, blockIdx.z, red);
+    absmax_body<DQK, HAD>(a.x[t], a.partial[t], a.N, a.H[t], a.nblk, blockIdx.y, h, blockIdx.z, red);
   else
-    absmax_body<DV, false>(a.x[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.x, h, blockIdx.z, red);
+    absmax_body<DV, false>(a.x[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.y, h, blockIdx.z, red);
 }
 
 template <int DQK, int DV, bool HAD, bool PER_HEAD>
 __global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_kernel(const QkvQuant a) {
   __shared__ float red[kQuantThreads / 32];
   int h;
-  const int t = qkv_pick(a, blockIdx.y, h);
+  const int t = qkv_pick(a, blockIdx.x, h);
   if (t < 2)
-    encode_body<DQK, HAD, PER_HEAD>(a.x[t], a.y[t], a.scale[t], a.partial[t], a.N, a.H[t], a.nblk, blockIdx.x, h,
+    encode_body<DQK, HAD, PER_HEAD>(a.x[t], a.y[t], a.scale[t], a.partial[t], a.N, a.H[t], a.nblk, blockIdx.y, h,
                                     blockIdx.z, red);
   else
-    encode_body<DV, false, PER_HEAD>(a.x[2], a.y[2], a.scale[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.x, h,
+    encode_body<DV, false, PER_HEAD>(a.x[2], a.y[2], a.scale[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.y, h,
                                      blockIdx.z, red);
 }
 

@@ -212,8 +212,8 @@ size_t b200attn_quantize_qkv_workspace_bytes(int B, int N, int Hq, int Hkv, int 
  *        (NULL allowed when that is 0); caller-owned, contents on entry do not
  *        matter, concurrent calls need distinct workspaces
  *
- * Errors: INVALID, UNSUPPORTED (head dims, more than 65535 heads in total),
- * WORKSPACE, CUDA.
+ * Errors: INVALID, UNSUPPORTED (head dims; N above 65535 blocks of 128 tokens,
+ * that is 8,388,480; B above 65535), WORKSPACE, CUDA.
  */
 int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v,
                               void* q_fp8, void* k_fp8, void* v_fp8,

@@ -135,7 +135,7 @@ def test_quantize_qkv_workspace_and_arguments_on_the_host(lib):
     assert qkv(lib, dqk=64) == -2
     assert qkv(lib, dv=192) == -2
     assert qkv(lib, gran=3) == -2
-    assert qkv(lib, Hq=65535, Hkv=1) == -2                  # more heads than a grid dimension holds
+    assert qkv(lib, N=65536 * 128) == -2                    # more token blocks than a grid dimension holds
     assert qkv(lib, ws=None) == -5
     assert qkv(lib, wsb=8) == -5
 
