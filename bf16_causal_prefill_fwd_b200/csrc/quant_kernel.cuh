@@ -253,6 +253,74 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_kernel(const Q
     absmax_body<DV, false>(a.x[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.y, h, blockIdx.z, red);
 }
 
+// Pass 1 over Q, K and V for d_qk = d_v = 128 on a persistent grid. CTA c takes
+// units c, c + gridDim.x, ... (a unit is one head's 128-token block, numbered
+// head fastest, then block, then batch) and issues the loads of its next unit
+// before it reduces the current one, so loads stay in flight while it reduces.
+// The maxima are those of quant_qkv_absmax_kernel, bit for bit.
+constexpr int kAbsmaxCtasPerSm = 2;
+
+__device__ __forceinline__ int qkv_unit(const QkvQuant& a, int u, int htot, int& h, int& blk, int& b) {
+  const int hidx = u % htot;
+  const int rest = u / htot;
+  blk = rest % a.nblk;
+  b = rest / a.nblk;
+  return qkv_pick(a, hidx, h);
+}
+
+// Raw bf16 pairs of this lane's 8 elements of the rows of one unit (d = 128).
+__device__ __forceinline__ void load_unit_raw(const QkvQuant& a, int u, int htot, int warp, int lane,
+                                              uint4 (&r)[QuantLayout<128>::ITERS]) {
+  using L = QuantLayout<128>;
+  int h, blk, b;
+  const int t = qkv_unit(a, u, htot, h, blk, b);
+  const __nv_bfloat16* x = a.x[t];
+  const int H = a.H[t], N = a.N;
+#pragma unroll
+  for (int it = 0; it < L::ITERS; ++it) {
+    const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + (lane >> 4);
+    const int rc = row < N ? row : N - 1;
+    r[it] = *reinterpret_cast<const uint4*>(x + (static_cast<size_t>(b) * N + rc) * H * 128 +
+                                            static_cast<size_t>(h) * 128 + 8 * (lane & 15));
+  }
+}
+
+template <bool HAD>
+__global__ void __launch_bounds__(kQuantThreads, kAbsmaxCtasPerSm)
+    quant_qkv_absmax_persistent_kernel(const QkvQuant a, int B) {
+  using L = QuantLayout<128>;
+  __shared__ float red[kQuantThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int htot = a.H[0] + a.H[1] + a.H[2];
+  const int total = htot * a.nblk * B;
+  int u = blockIdx.x;
+  if (u >= total) return;  // the same for every thread of the CTA
+  uint4 cur[L::ITERS], nxt[L::ITERS];
+  load_unit_raw(a, u, htot, warp, lane, cur);
+  for (; u < total; u += gridDim.x) {
+    const int un = u + gridDim.x;
+    if (un < total) load_unit_raw(a, un, htot, warp, lane, nxt);
+    int h, blk, b;
+    const int t = qkv_unit(a, u, htot, h, blk, b);
+    float m = 0.0f;
+#pragma unroll
+    for (int it = 0; it < L::ITERS; ++it) {
+      float v[8];
+      bf16x8_to_float(cur[it], v);
+      if (HAD && t < 2) rotate_lane<128>(lane, v);  // t is the same for the whole CTA
+      const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + (lane >> 4);
+      if (row < a.N) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+      }
+    }
+    m = block_max(m, red);
+    if (threadIdx.x == 0) a.partial[t][(static_cast<size_t>(b) * a.H[t] + h) * a.nblk + blk] = m;
+#pragma unroll
+    for (int it = 0; it < L::ITERS; ++it) cur[it] = nxt[it];
+  }
+}
+
 template <int DQK, int DV, bool HAD, bool PER_HEAD>
 __global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_kernel(const QkvQuant a) {
   __shared__ float red[kQuantThreads / 32];

@@ -54,7 +54,10 @@ def test_full_size_q_bit_exact(name, hadamard):
         assert np.array_equal(codes, ref_codes)
 
 
-@pytest.mark.parametrize("shape", [(1, 300, 4, 2, 128), (2, 129, 2, 2, 192), (1, 1000, 8, 1, 128)])
+# (2, 4000, 8, 2, 128) has more 128-token head blocks (768) than the persistent
+# per-head amax pass has CTAs, so each CTA loops over several.
+@pytest.mark.parametrize("shape", [(1, 300, 4, 2, 128), (2, 129, 2, 2, 192), (1, 1000, 8, 1, 128),
+                                   (2, 4000, 8, 2, 128)])
 @pytest.mark.parametrize("granularity", ["head", "block"])
 @pytest.mark.parametrize("hadamard", [False, True])
 def test_qkv_in_one_launch_bit_exact(shape, granularity, hadamard):
@@ -71,3 +74,22 @@ def test_qkv_in_one_launch_bit_exact(shape, granularity, hadamard):
         ref_codes, ref_scale = oracle.quantize_fp8(f32(t), granularity, rot)
         assert np.array_equal(s.cpu().numpy(), ref_scale)
         assert np.array_equal(c.view(torch.uint8).cpu().numpy(), ref_codes)
+
+
+@pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("qknorm", True)])
+def test_full_size_qkv_bit_exact(name, hadamard):
+    """The merged quantizer at full size, in the launch configuration of the FP8
+    step: K and V equal the oracle's codes and scales; Q equals the per-tensor
+    quantizer's (pinned to the oracle above), which keeps the oracle off the
+    64 Mi-element Q."""
+    w = workloads.BY_NAME[name]()
+    q, k, v = workloads.draw(w)
+    outs = b2.quantize_qkv_fp8(q.cuda(), k.cuda(), v.cuda(), hadamard=hadamard)
+    assert b2.check() == 0
+    for t, rot, (c, s) in ((k, hadamard, outs[2:4]), (v, False, outs[4:6])):
+        ref_codes, ref_scale = oracle.quantize_fp8(f32(t), "head", rot)
+        assert np.array_equal(s.cpu().numpy(), ref_scale)
+        assert np.array_equal(c.view(torch.uint8).cpu().numpy(), ref_codes)
+    q_codes, q_scale = gpu_quant(q, "head", hadamard)
+    assert np.array_equal(outs[1].cpu().numpy(), q_scale)
+    assert np.array_equal(outs[0].view(torch.uint8).cpu().numpy(), q_codes)
