@@ -164,14 +164,14 @@ int launch_quant(const void* x, void* y, float* scale, int B, int N, int H, int 
 }
 
 template <int DQK, int DV, bool HAD>
-int launch_quant_qkv(const b200::QkvQuant& a, int B, int gran, int sm_count, cudaStream_t stream) {
+int launch_quant_qkv(const b200::QkvQuant& a, int B, int gran, cudaStream_t stream) {
   const dim3 grid(a.H[0] + a.H[1] + a.H[2], a.nblk, B);
-  const int64_t units = static_cast<int64_t>(grid.x) * grid.y * grid.z;
   if (gran == B200ATTN_SCALE_PER_HEAD) {
-    if (DQK == 128 && DV == 128 && units < (int64_t(1) << 31)) {
-      const int ctas = sm_count * b200::kAbsmaxCtasPerSm;
-      b200::quant_qkv_absmax_persistent_kernel<HAD>
-          <<<units < ctas ? static_cast<int>(units) : ctas, b200::kQuantThreads, 0, stream>>>(a, B);
+    if (DQK == 128 && DV == 128 && a.H[0] % 2 == 0 && a.H[1] % 2 == 0) {
+      const dim3 ggrid(grid.x / 2, a.nblk, B);
+      b200::quant_qkv_absmax_group_kernel<HAD, 2><<<ggrid, b200::kQuantThreads, 0, stream>>>(a);
+    } else if (DQK == 128 && DV == 128) {
+      b200::quant_qkv_absmax_group_kernel<HAD, 1><<<grid, b200::kQuantThreads, 0, stream>>>(a);
     } else {
       b200::quant_qkv_absmax_kernel<DQK, DV, HAD><<<grid, b200::kQuantThreads, 0, stream>>>(a);
     }
@@ -454,10 +454,10 @@ int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v, void*
   a.partial[2] = ws ? ws + static_cast<size_t>(B) * (Hq + Hkv) * nblk : nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d_qk == 128)
-    return hadamard ? launch_quant_qkv<128, 128, true>(a, B, granularity, sm_count, st)
-                    : launch_quant_qkv<128, 128, false>(a, B, granularity, sm_count, st);
-  return hadamard ? launch_quant_qkv<192, 128, true>(a, B, granularity, sm_count, st)
-                  : launch_quant_qkv<192, 128, false>(a, B, granularity, sm_count, st);
+    return hadamard ? launch_quant_qkv<128, 128, true>(a, B, granularity, st)
+                    : launch_quant_qkv<128, 128, false>(a, B, granularity, st);
+  return hadamard ? launch_quant_qkv<192, 128, true>(a, B, granularity, st)
+                  : launch_quant_qkv<192, 128, false>(a, B, granularity, st);
 }
 
 

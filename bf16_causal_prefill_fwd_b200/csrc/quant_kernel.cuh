@@ -8,7 +8,9 @@
 // 开源 ZYFA …", "ZYFA 的 FP8 注意力有多准确？" (a Hadamard rotation of Q and K
 // roughly halves the input-quantisation error at ~0.1% attention time).
 //
-// HBM-bound: one CTA of 8 warps per (b, h, 128-token block). A row is held by
+// HBM-bound: one CTA of 8 warps per (b, h, 128-token block), except the d = 128
+// absmax pass over Q, K and V, which takes a pair of heads per CTA (see
+// quant_qkv_absmax_group_kernel). A row is held by
 // 16 lanes: for d = 128 each lane loads 8 bf16 (16 bytes), so one warp
 // instruction moves two rows; for d = 192 lanes 0-15 load 8 of the first 128
 // and lanes 16-31 load 4 of the 64-wide tail. Every load of the block is
@@ -253,71 +255,74 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_kernel(const Q
     absmax_body<DV, false>(a.x[2], a.partial[2], a.N, a.H[2], a.nblk, blockIdx.y, h, blockIdx.z, red);
 }
 
-// Pass 1 over Q, K and V for d_qk = d_v = 128 on a persistent grid. CTA c takes
-// units c, c + gridDim.x, ... (a unit is one head's 128-token block, numbered
-// head fastest, then block, then batch) and issues the loads of its next unit
-// before it reduces the current one, so loads stay in flight while it reduces.
+// Pass 1 over Q, K and V for d_qk = d_v = 128, one CTA per (tensor, group of G
+// consecutive heads, 128-token block): blockIdx.x walks the head groups of Q,
+// then K, then V; blockIdx.y the blocks. A row of the group is G*256 contiguous
+// bytes. Each step the 256 threads load 4 KiB of consecutive rows, 8 steps in
+// flight; a half-warp always holds one 128-wide head row (its 16-byte segment
+// is lane & 15), which is the layout of the rotation, and thread t always sees
+// head (t mod 16G) / 16 of the group.
 // The maxima are those of quant_qkv_absmax_kernel, bit for bit.
-constexpr int kAbsmaxCtasPerSm = 2;
-
-__device__ __forceinline__ int qkv_unit(const QkvQuant& a, int u, int htot, int& h, int& blk, int& b) {
-  const int hidx = u % htot;
-  const int rest = u / htot;
-  blk = rest % a.nblk;
-  b = rest / a.nblk;
-  return qkv_pick(a, hidx, h);
+template <typename T>
+__device__ __forceinline__ T pick3(const T (&arr)[3], int t) {  // no dynamic index into the parameters
+  return t == 0 ? arr[0] : (t == 1 ? arr[1] : arr[2]);
 }
 
-// Raw bf16 pairs of this lane's 8 elements of the rows of one unit (d = 128).
-__device__ __forceinline__ void load_unit_raw(const QkvQuant& a, int u, int htot, int warp, int lane,
-                                              uint4 (&r)[QuantLayout<128>::ITERS]) {
-  using L = QuantLayout<128>;
-  int h, blk, b;
-  const int t = qkv_unit(a, u, htot, h, blk, b);
-  const __nv_bfloat16* x = a.x[t];
-  const int H = a.H[t], N = a.N;
-#pragma unroll
-  for (int it = 0; it < L::ITERS; ++it) {
-    const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + (lane >> 4);
-    const int rc = row < N ? row : N - 1;
-    r[it] = *reinterpret_cast<const uint4*>(x + (static_cast<size_t>(b) * N + rc) * H * 128 +
-                                            static_cast<size_t>(h) * 128 + 8 * (lane & 15));
+template <bool HAD, int G>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_kernel(const QkvQuant a) {
+  constexpr int kChunks = 16 * G;             // 16-byte segments in a row of the group
+  constexpr int kRowsPerStep = kQuantThreads / kChunks;
+  constexpr int kSteps = kQuantBlock / kRowsPerStep;
+  static_assert(kSteps % 8 == 0, "steps are loaded eight at a time");
+  __shared__ float red[kQuantThreads / 32][2];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = a.H[0] / G, gk = a.H[1] / G;
+  int t, g = blockIdx.x;
+  if (g < gq) {
+    t = 0;
+  } else if (g < gq + gk) {
+    t = 1;
+    g -= gq;
+  } else {
+    t = 2;
+    g -= gq + gk;
   }
-}
-
-template <bool HAD>
-__global__ void __launch_bounds__(kQuantThreads, kAbsmaxCtasPerSm)
-    quant_qkv_absmax_persistent_kernel(const QkvQuant a, int B) {
-  using L = QuantLayout<128>;
-  __shared__ float red[kQuantThreads / 32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int htot = a.H[0] + a.H[1] + a.H[2];
-  const int total = htot * a.nblk * B;
-  int u = blockIdx.x;
-  if (u >= total) return;  // the same for every thread of the CTA
-  uint4 cur[L::ITERS], nxt[L::ITERS];
-  load_unit_raw(a, u, htot, warp, lane, cur);
-  for (; u < total; u += gridDim.x) {
-    const int un = u + gridDim.x;
-    if (un < total) load_unit_raw(a, un, htot, warp, lane, nxt);
-    int h, blk, b;
-    const int t = qkv_unit(a, u, htot, h, blk, b);
-    float m = 0.0f;
+  const int H = pick3(a.H, t), N = a.N, blk = blockIdx.y, b = blockIdx.z;
+  const int r_in = tid / kChunks;
+  const uint4* base = reinterpret_cast<const uint4*>(pick3(a.x, t)) + static_cast<size_t>(b) * N * H * 16 +
+                      static_cast<size_t>(g) * kChunks + tid % kChunks;
+  float m = 0.0f;
+#pragma unroll 1
+  for (int s0 = 0; s0 < kSteps; s0 += 8) {
+    uint4 r[8];
 #pragma unroll
-    for (int it = 0; it < L::ITERS; ++it) {
+    for (int k = 0; k < 8; ++k) {
+      const int row = blk * kQuantBlock + (s0 + k) * kRowsPerStep + r_in;
+      r[k] = base[static_cast<size_t>(row < N ? row : N - 1) * H * 16];
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
       float v[8];
-      bf16x8_to_float(cur[it], v);
+      bf16x8_to_float(r[k], v);
       if (HAD && t < 2) rotate_lane<128>(lane, v);  // t is the same for the whole CTA
-      const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + (lane >> 4);
-      if (row < a.N) {
+      if (blk * kQuantBlock + (s0 + k) * kRowsPerStep + r_in < N) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
       }
     }
-    m = block_max(m, red);
-    if (threadIdx.x == 0) a.partial[t][(static_cast<size_t>(b) * a.H[t] + h) * a.nblk + blk] = m;
+  }
 #pragma unroll
-    for (int it = 0; it < L::ITERS; ++it) cur[it] = nxt[it];
+  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));  // within a half-warp
+  if ((lane & 15) == 0) red[warp][lane >> 4] = m;
+  __syncthreads();
+  if (tid < G) {  // head tid of the group
+    float mh = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kQuantThreads / 32; ++w)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        if (((w * 32 + hh * 16) % kChunks) / 16 == tid) mh = fmaxf(mh, red[w][hh]);
+    pick3(a.partial, t)[(static_cast<size_t>(b) * H + g * G + tid) * a.nblk + blk] = mh;
   }
 }
 
