@@ -326,6 +326,99 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_kernel(c
   }
 }
 
+// Pass 2 (per-head scales) over Q, K and V for d_qk = d_v = 128, on the grid and
+// thread layout of quant_qkv_absmax_group_kernel. The scale of a head comes
+// from its partial maxima alone, so the block's rows stream through: eight
+// loads in flight, then rotate, scale, convert and store them, eight steps at a
+// time. The first loads are issued before the partial maxima are reduced.
+// Codes and scales are those of quant_qkv_encode_kernel, bit for bit.
+template <bool HAD, int G>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_group_kernel(const QkvQuant a) {
+  constexpr int kChunks = 16 * G;
+  constexpr int kRowsPerStep = kQuantThreads / kChunks;
+  constexpr int kSteps = kQuantBlock / kRowsPerStep;
+  static_assert(kSteps % 8 == 0, "steps are loaded eight at a time");
+  __shared__ float red[kQuantThreads / 32][G];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = a.H[0] / G, gk = a.H[1] / G;
+  int t, g = blockIdx.x;
+  if (g < gq) {
+    t = 0;
+  } else if (g < gq + gk) {
+    t = 1;
+    g -= gq;
+  } else {
+    t = 2;
+    g -= gq + gk;
+  }
+  const int H = pick3(a.H, t), N = a.N, blk = blockIdx.y, b = blockIdx.z;
+  const int r_in = tid / kChunks, hl = (tid % kChunks) / 16;
+  const size_t first = static_cast<size_t>(b) * N * H * 16 + static_cast<size_t>(g) * kChunks + tid % kChunks;
+  const uint4* src = reinterpret_cast<const uint4*>(pick3(a.x, t)) + first;
+  uint2* dst = reinterpret_cast<uint2*>(pick3(a.y, t)) + first;  // an e4m3 row is H*16 uint2
+
+  uint4 r[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int row = blk * kQuantBlock + k * kRowsPerStep + r_in;
+    r[k] = src[static_cast<size_t>(row < N ? row : N - 1) * H * 16];
+  }
+
+  // amax of each head of the group: the max of its partials
+  const float* ph = pick3(a.partial, t) + (static_cast<size_t>(b) * H + g * G) * a.nblk;
+  float mh[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    mh[j] = 0.0f;
+    for (int i = tid; i < a.nblk; i += kQuantThreads) mh[j] = fmaxf(mh[j], ph[static_cast<size_t>(j) * a.nblk + i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mh[j] = fmaxf(mh[j], __shfl_xor_sync(0xffffffffu, mh[j], o));
+    if (lane == 0) red[warp][j] = mh[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    mh[j] = red[0][j];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) mh[j] = fmaxf(mh[j], red[w][j]);
+  }
+  float amax = mh[0];
+#pragma unroll
+  for (int j = 1; j < G; ++j) amax = hl == j ? mh[j] : amax;
+  const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  if (blk == 0 && tid < G) {
+    float as = mh[0];
+#pragma unroll
+    for (int j = 1; j < G; ++j) as = tid == j ? mh[j] : as;
+    pick3(a.scale, t)[static_cast<size_t>(b) * H + g * G + tid] = as > 0.0f ? __fdiv_rn(as, 448.0f) : 1.0f;
+  }
+
+#pragma unroll 1
+  for (int s0 = 0; s0 < kSteps; s0 += 8) {
+    if (s0 > 0) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int row = blk * kQuantBlock + (s0 + k) * kRowsPerStep + r_in;
+        r[k] = src[static_cast<size_t>(row < N ? row : N - 1) * H * 16];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float v[8];
+      bf16x8_to_float(r[k], v);
+      if (HAD && t < 2) rotate_lane<128>(lane, v);  // t is the same for the whole CTA
+      const int row = blk * kQuantBlock + (s0 + k) * kRowsPerStep + r_in;
+      if (row < N) {
+        uint32_t c[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          c[q] = pack_e4m3x2(__fmul_rn(v[2 * q], inv), __fmul_rn(v[2 * q + 1], inv));
+        dst[static_cast<size_t>(row) * H * 16] = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+      }
+    }
+  }
+}
+
 template <int DQK, int DV, bool HAD, bool PER_HEAD>
 __global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_kernel(const QkvQuant a) {
   __shared__ float red[kQuantThreads / 32];
