@@ -17,6 +17,7 @@
 // issued before any arithmetic (row indices are clamped, never branched on),
 // which keeps 32 KiB per CTA in flight. The rotated values stay in registers
 // between the absmax reduction and the encode, so x is read once per pass.
+// The d = 128 head-group kernels further down stream rows through instead.
 //
 // Arithmetic contract (identical on every call, so codes are reproducible):
 //   rotation: radix-2 butterflies of widths 1, 2, 4, ... (the lower element of
