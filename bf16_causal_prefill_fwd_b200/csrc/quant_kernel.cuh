@@ -9,7 +9,7 @@
 // roughly halves the input-quantisation error at ~0.1% attention time).
 //
 // HBM-bound: one CTA of 8 warps per (b, h, 128-token block), except the d = 128
-// absmax pass over Q, K and V, which takes a pair of heads per CTA (see
+// per-head passes over Q, K and V, which take a group of heads per CTA (see
 // quant_qkv_absmax_group_kernel). A row is held by
 // 16 lanes: for d = 128 each lane loads 8 bf16 (16 bytes), so one warp
 // instruction moves two rows; for d = 192 lanes 0-15 load 8 of the first 128
