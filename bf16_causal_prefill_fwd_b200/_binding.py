@@ -91,6 +91,43 @@ def _is_fp8(t):
     return t.dtype in (torch.float8_e4m3fn, torch.uint8)
 
 
+_E4M3_DTYPES = (torch.float8_e4m3fn, torch.uint8)
+
+
+def _check_buffer(name, t, shape, dtypes, device):
+    """A caller-supplied buffer the kernels read or write in full: it must be a
+    contiguous CUDA tensor on ``device`` with exactly ``shape`` elements laid out
+    as documented, else the kernels would run past its end."""
+    _check_cuda_contig(name, t)
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must have dtype {' or '.join(str(d) for d in dtypes)}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _gran(granularity: str) -> int:
+    if granularity not in _GRAN:
+        raise ValueError("granularity must be 'head' or 'block'")
+    return _GRAN[granularity]
+
+
+def _scale_shape(B: int, H: int, N: int, granularity: str):
+    return (B, H) if granularity == "head" else (B, H, math.ceil(N / BLOCK))
+
+
+def _check_scale(name, s, B, H, N, granularity, device):
+    """fp32 scales [B, H] (per head) or [B, H, ceil(N/128)] (per block); a flat
+    tensor with that many elements is accepted too."""
+    if s is None:
+        raise ValueError(f"{name} is required for e4m3 inputs")
+    shape = _scale_shape(B, H, N, granularity)
+    if isinstance(s, torch.Tensor) and s.dim() == 1 and s.numel() == math.prod(shape):
+        shape = (s.numel(),)
+    _check_buffer(name, s, shape, (torch.float32,), device)
+
+
 def attn_fwd(q, k, v, *, causal: bool = True, softmax_scale: float | None = None,
              q_scale=None, k_scale=None, v_scale=None, scale_granularity: str = "head",
              out=None, return_lse: bool = False, stream=None):
@@ -112,25 +149,23 @@ def attn_fwd(q, k, v, *, causal: bool = True, softmax_scale: float | None = None
     Hkv, d_v = k.shape[2], v.shape[3]
     if k.shape != (B, N, Hkv, d_qk) or v.shape != (B, N, Hkv, d_v):
         raise ValueError("shape mismatch between q, k and v")
+    gran = _gran(scale_granularity)
+    dev = q.device
+    if k.device != dev or v.device != dev:
+        raise ValueError("q, k and v must be on one device")
     if out is None:
-        out = torch.empty((B, N, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((B, N, Hq, d_v), dtype=torch.bfloat16, device=dev)
     else:
-        _check_cuda_contig("out", out)
-        if out.dtype != torch.bfloat16 or out.shape != (B, N, Hq, d_v):
-            raise ValueError("out must be bf16 [B, N, Hq, d_v]")
-    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if return_lse else None
+        _check_buffer("out", out, (B, N, Hq, d_v), (torch.bfloat16,), dev)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev) if return_lse else None
     if fp8:
-        for name, s in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
-            if s is None:
-                raise ValueError(f"{name} is required for e4m3 inputs")
-            _check_cuda_contig(name, s)
-            if s.dtype != torch.float32:
-                raise ValueError(f"{name} must be fp32")
+        for name, sc, H in (("q_scale", q_scale, Hq), ("k_scale", k_scale, Hkv), ("v_scale", v_scale, Hkv)):
+            _check_scale(name, sc, B, H, N, scale_granularity, dev)
     rc = lib.b200attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, N, d_qk, d_v, 1 if causal else 0,
         FP8_E4M3 if fp8 else BF16,
         _ptr(q_scale) if fp8 else None, _ptr(k_scale) if fp8 else None, _ptr(v_scale) if fp8 else None,
-        _GRAN[scale_granularity], float(softmax_scale) if softmax_scale else 0.0,
+        gran, float(softmax_scale) if softmax_scale else 0.0,
         _ptr(lse), _stream_handle(stream))
     if rc != 0:
         raise B200AttnError(rc, "b200attn_fwd")
@@ -162,18 +197,23 @@ def attn_varlen_fwd(q, k, v, cu_seqlens, *, causal: bool = True, softmax_scale: 
     if k.shape != (total, Hkv, d_qk) or v.shape != (total, Hkv, d_v):
         raise ValueError("shape mismatch between q, k and v")
     cu, batch = _cu_array(cu_seqlens)
+    dev = q.device
+    if k.device != dev or v.device != dev:
+        raise ValueError("q, k and v must be on one device")
     if out is None:
-        out = torch.empty((total, Hq, d_v), dtype=torch.bfloat16, device=q.device)
-    lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device) if return_lse else None
+        out = torch.empty((total, Hq, d_v), dtype=torch.bfloat16, device=dev)
+    else:
+        _check_buffer("out", out, (total, Hq, d_v), (torch.bfloat16,), dev)
+    lse = torch.empty((Hq, total), dtype=torch.float32, device=dev) if return_lse else None
     if total == 0:  # nothing to compute (and no device memory to point at)
         if batch < 1 or any(c != 0 for c in cu):
             raise ValueError("cu_seqlens must be non-decreasing from 0 to total")
         return (out, lse) if return_lse else out
     if fp8:
-        for name, sc in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+        for name, sc, H in (("q_scale", q_scale, Hq), ("k_scale", k_scale, Hkv), ("v_scale", v_scale, Hkv)):
             if sc is None:
                 raise ValueError(f"{name} is required for e4m3 inputs")
-            _check_cuda_contig(name, sc)
+            _check_buffer(name, sc, (H,) if sc.dim() == 1 else (1, H), (torch.float32,), dev)
     need = int(lib.b200attn_fwd_varlen_workspace_bytes(cu, batch, Hq))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -201,7 +241,7 @@ def attn_varlen_func(q, k, v, cu_seqlens, softmax_scale: float | None = None, ca
 
 
 def quantize_workspace_bytes(B, N, H, d, granularity="head") -> int:
-    return int(load_library().b200attn_quantize_workspace_bytes(B, N, H, d, _GRAN[granularity]))
+    return int(load_library().b200attn_quantize_workspace_bytes(B, N, H, d, _gran(granularity)))
 
 
 def quantize_fp8(x, *, granularity: str = "head", hadamard: bool = False, out=None, scale=None,
@@ -216,16 +256,20 @@ def quantize_fp8(x, *, granularity: str = "head", hadamard: bool = False, out=No
     if x.dtype != torch.bfloat16 or x.dim() != 4:
         raise ValueError("x must be bf16 [B, N, H, d]")
     B, N, H, d = x.shape
+    gran = _gran(granularity)
     if out is None:
         out = torch.empty((B, N, H, d), dtype=torch.float8_e4m3fn, device=x.device)
+    else:
+        _check_buffer("out", out, (B, N, H, d), _E4M3_DTYPES, x.device)
     if scale is None:
-        shape = (B, H) if granularity == "head" else (B, H, math.ceil(N / BLOCK))
-        scale = torch.empty(shape, dtype=torch.float32, device=x.device)
+        scale = torch.empty(_scale_shape(B, H, N, granularity), dtype=torch.float32, device=x.device)
+    else:
+        _check_buffer("scale", scale, _scale_shape(B, H, N, granularity), (torch.float32,), x.device)
     need = quantize_workspace_bytes(B, N, H, d, granularity)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.b200attn_quantize_fp8(_ptr(x), _ptr(out), _ptr(scale), B, N, H, d, _GRAN[granularity],
+    rc = lib.b200attn_quantize_fp8(_ptr(x), _ptr(out), _ptr(scale), B, N, H, d, gran,
                                    1 if hadamard else 0, _ptr(workspace), wbytes, _stream_handle(stream))
     if rc != 0:
         raise B200AttnError(rc, "b200attn_quantize_fp8")
@@ -233,7 +277,7 @@ def quantize_fp8(x, *, granularity: str = "head", hadamard: bool = False, out=No
 
 
 def quantize_qkv_workspace_bytes(B, N, Hq, Hkv, granularity="head") -> int:
-    return int(load_library().b200attn_quantize_qkv_workspace_bytes(B, N, Hq, Hkv, _GRAN[granularity]))
+    return int(load_library().b200attn_quantize_qkv_workspace_bytes(B, N, Hq, Hkv, _gran(granularity)))
 
 
 def quantize_qkv_fp8(q, k, v, *, granularity: str = "head", hadamard: bool = False, out=None, workspace=None,
@@ -250,20 +294,28 @@ def quantize_qkv_fp8(q, k, v, *, granularity: str = "head", hadamard: bool = Fal
     Hkv, d_v = k.shape[2], v.shape[3]
     if k.shape != (B, N, Hkv, d_qk) or v.shape != (B, N, Hkv, d_v):
         raise ValueError("shape mismatch between q, k and v")
+    gran = _gran(granularity)
+    dev = q.device
+    if k.device != dev or v.device != dev:
+        raise ValueError("q, k and v must be on one device")
     if out is None:
-        nb = math.ceil(N / BLOCK)
-        dev = q.device
         out = []
         for t, H in ((q, Hq), (k, Hkv), (v, Hkv)):
             out.append(torch.empty(t.shape, dtype=torch.float8_e4m3fn, device=dev))
-            out.append(torch.empty((B, H) if granularity == "head" else (B, H, nb), dtype=torch.float32, device=dev))
+            out.append(torch.empty(_scale_shape(B, H, N, granularity), dtype=torch.float32, device=dev))
+    else:
+        if len(out) != 6:
+            raise ValueError("out must hold six tensors: q8, q_scale, k8, k_scale, v8, v_scale")
+        for i, (name, t, H) in enumerate((("q", q, Hq), ("k", k, Hkv), ("v", v, Hkv))):
+            _check_buffer(f"{name}8", out[2 * i], tuple(t.shape), _E4M3_DTYPES, dev)
+            _check_buffer(f"{name}_scale", out[2 * i + 1], _scale_shape(B, H, N, granularity), (torch.float32,), dev)
     q8, sq, k8, sk, v8, sv = out
     need = quantize_qkv_workspace_bytes(B, N, Hq, Hkv, granularity)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = lib.b200attn_quantize_qkv_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk),
-                                       _ptr(sv), B, N, Hq, Hkv, d_qk, d_v, _GRAN[granularity],
+                                       _ptr(sv), B, N, Hq, Hkv, d_qk, d_v, gran,
                                        1 if hadamard else 0, _ptr(workspace), wbytes, _stream_handle(stream))
     if rc != 0:
         raise B200AttnError(rc, "b200attn_quantize_qkv_fp8")
