@@ -337,6 +337,21 @@ def measure_energy(clk, path, flops_per_step: float, seconds: float):
             "source": "NVML total energy consumption of this GPU over steps run back to back (no L2 flush)"}
 
 
+def quantizer_summary(quant_ms: float, w: workloads.Workload, hbm_peak: float) -> dict:
+    """The FP8 step's quantizer against the HBM roofline. quant_ms is the part of the step
+    outside the attention kernel's events: the absmax and encode launches plus launch gaps.
+    Algorithmic bytes with per-head scales: a 2-byte read in each pass and a 1-byte write,
+    5 bytes per element of Q, K and V."""
+    elems = w.B * w.N * (w.Hq * w.d_qk + w.Hkv * (w.d_qk + w.d_v))
+    nbytes = 5.0 * elems
+    if not quant_ms > 0.0:
+        return None
+    gbs = nbytes / (quant_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "ms": quant_ms, "algorithmic_bytes": nbytes, "achieved": gbs, "unit": "GB/s",
+            "peak": hbm_peak, "frac": gbs / hbm_peak,
+            "timed": "step time outside the attention kernel's CUDA events (quantizer launches and gaps)"}
+
+
 def max_over_ranks(x: float, dist_on: bool, device: str = "cuda") -> float:
     """The slowest rank's value: every rank contributes its own timing, all get the max."""
     if not dist_on:
@@ -357,6 +372,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     peaks, peak_src = load_peaks()
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
     def measure(dtype, clk=None):
         path = Path(b2, q, k, v, dtype, args.hadamard)
@@ -379,7 +395,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "peak_source": (f"{peak_src} bf16 burst {bf16_peak} TFLOP/s"
                                 + (" x2 (nominal fp8/bf16 ratio 4.5/2.25)" if dtype == "fp8" else "")),
                 "frac_of_spec_dense": achieved / (4500.0 if dtype == "fp8" else 2250.0)}
-        return {"value": value, "ms_per_step": ms, "roofline": roof,
+        quant = None
+        if dtype == "fp8":
+            qms = max_over_ranks(statistics.mean([s - a for s, a in zip(step_ms, attn_ms)]), dist_on)
+            quant = quantizer_summary(qms, w, hbm_peak)
+        return {"value": value, "ms_per_step": ms, "roofline": roof, "quantizer": quant,
                 "launches": path.launches_per_step * args.steps,
                 "step_ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))]}
 
@@ -421,6 +441,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                   if args.dtype == "bf16" else None),
                        "parallelism": f"replicas x{world}"},
             "roofline": main["roofline"],
+            "quantizer": main["quantizer"],
             "clocks": clocks,
             "energy": energy,
             "gpu_launches": main["launches"],

@@ -1,5 +1,6 @@
-"""The N>1 plumbing of bench.py on CPU with gloo (world size 2): every rank
-gets the slowest rank's time, and the reference arm runs on rank 0 only."""
+"""bench.py host logic on CPU. The N>1 plumbing with gloo (world size 2): every rank
+gets the slowest rank's time, and the reference arm runs on rank 0 only. Also the
+quantizer's HBM-roofline arithmetic."""
 import os
 import socket
 
@@ -49,3 +50,18 @@ def test_reference_arm_other_ranks_do_no_work(capsys):
         workload, n, warmup, steps = "tiny", None, 3, 1
     bench.run_reference(A(), rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+def test_quantizer_summary_counts_five_bytes_per_element():
+    """Per-head scales: the absmax pass reads 2 bytes, the encode pass reads 2 and
+    writes 1, over every element of Q, K and V."""
+    import bench
+    import workloads
+    w = workloads.gqa7b()
+    s = bench.quantizer_summary(0.1, w, 6545.3)
+    assert s["algorithmic_bytes"] == 5 * (32 + 8 + 8) * 128 * 16384
+    assert abs(s["achieved"] - s["algorithmic_bytes"] / 1e-4 / 1e9) < 1e-6
+    assert abs(s["frac"] - s["achieved"] / 6545.3) < 1e-12 and s["bound"] == "hbm"
+    m = bench.quantizer_summary(0.1, workloads.mla(), 6545.3)
+    assert m["algorithmic_bytes"] == 5 * 16 * (192 + 192 + 128) * 16384
+    assert bench.quantizer_summary(0.0, w, 6545.3) is None
