@@ -76,6 +76,9 @@ def test_fwd_reports_unsupported_shapes_on_the_host(lib):
     assert fwd(lib, dqk=128, dv=192) == -2
     assert fwd(lib, dtype=7) == -2
     assert fwd(lib, dtype=1, qs=FAKE, ks=FAKE, vs=FAKE, gran=5) == -2
+    # the kernels index (b, n, h) rows in 32 bits: B*N*max(Hq, Hkv) must stay below 2^31
+    assert fwd(lib, B=1, N=1 << 26, Hq=32, Hkv=8) == -2
+    assert fwd(lib, B=1 << 10, N=1 << 16, Hq=32, Hkv=8) == -2
 
 
 def test_quantize_workspace_size(lib):
@@ -95,6 +98,8 @@ def test_quantize_rejects_bad_arguments_on_the_host(lib):
     assert q(FAKE + 4, FAKE, FAKE, 1, 10, 1, 128, 0, 0, FAKE, 64, None) == -1
     assert q(FAKE, FAKE, FAKE, 1, 10, 1, 128, 0, 0, None, 0, None) == -5     # per-head needs a workspace
     assert q(FAKE, FAKE, FAKE, 1, 300, 2, 128, 0, 0, FAKE, 8, None) == -5    # too small
+    assert q(FAKE, FAKE, FAKE, 1, 300, 65536, 128, 1, 0, None, 0, None) == -2  # more heads than a grid dimension
+    assert q(FAKE, FAKE, FAKE, 65536, 300, 1, 128, 1, 0, None, 0, None) == -2  # batch beyond a grid dimension
 
 
 def test_binding_refuses_cpu_tensors():
