@@ -161,3 +161,43 @@ def test_varlen_workspace_and_arguments_on_the_host(lib):
     assert call([0, 100, 400], 400, dtype=1) == -1   # FP8 without scales
     assert call([0, 100, 400], 400, ws=None) == -5
     assert call([0, 100, 400], 400, wsb=16) == -5
+
+
+def header_prototypes():
+    """{name: (return C type, [parameter C types])} for every entry point in the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for ret, name, params in re.findall(r"((?:const\s+)?\w+\s*\**)\s*(b200attn_\w+)\s*\(([^)]*)\)\s*;", text):
+        types = []
+        for p in params.split(","):
+            p = " ".join(p.split())
+            if not p or p == "void":
+                continue
+            types.append(re.sub(r"\s*\b\w+$", "", p).replace(" *", "*"))   # drop the parameter name
+        protos[name] = (" ".join(ret.split()).replace(" *", "*"), types)
+    return protos
+
+
+def ctype_of(c):
+    if c.endswith("*"):
+        base = c.replace("const", "").replace("*", "").strip()
+        if base == "char":
+            return ctypes.c_char_p
+        return ctypes.POINTER(ctypes.c_int) if base == "int" else ctypes.c_void_p
+    return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t}[c]
+
+
+def test_binding_argtypes_match_header_prototypes(lib):
+    """Every entry point the binding declares to ctypes has the header's parameter list:
+    a wrong count or type would pass garbage to the library without an error."""
+    protos = header_prototypes()
+    assert set(protos) == set(declared_functions())
+    checked = 0
+    for name, (ret, params) in protos.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is None:
+            continue  # not declared by the binding (called only through raw ctypes in tests)
+        assert list(fn.argtypes) == [ctype_of(p) for p in params], name
+        assert fn.restype == ctype_of(ret), name
+        checked += 1
+    assert checked >= 10
