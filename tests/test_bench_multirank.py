@@ -65,3 +65,23 @@ def test_quantizer_summary_counts_five_bytes_per_element():
     m = bench.quantizer_summary(0.1, workloads.mla(), 6545.3)
     assert m["algorithmic_bytes"] == 5 * 16 * (192 + 192 + 128) * 16384
     assert bench.quantizer_summary(0.0, w, 6545.3) is None
+
+
+def test_reference_arm_line_on_rank_zero(capsys):
+    """The reference arm's JSON line: the oracle on a bounded sample, the same workload
+    string as the GPU arm, and the keys the line must carry."""
+    import json
+    import bench
+
+    class A:
+        workload, n, warmup, steps = "tiny", None, 3, 1
+    bench.run_reference(A(), rank=0, world=1)
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == bench.workload_desc(bench.make_workload("tiny", None))
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["dtype"] == "f64"
