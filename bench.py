@@ -94,7 +94,7 @@ def kernel_sources_sha() -> str:
 def traffic_for(kernel_key: str, workload_name: str):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the
     current kernel source; otherwise None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic_gqa7b.json")
     try:
         with open(path) as f:
             d = json.load(f)
