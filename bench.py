@@ -63,6 +63,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-dtype", action="store_true", help="skip the secondary dtype measurement")
+    ap.add_argument("--no-at-32k", action="store_true", help="skip the N=32768 (B=1) Gaussian layer")
+    ap.add_argument("--measure-peaks", action="store_true",
+                    help="print the bf16 and e4m3 GEMM tensor peaks of this GPU as JSON and exit")
     return ap.parse_args()
 
 
@@ -175,6 +178,78 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------
+# tensor-core peaks of library GEMMs on this GPU (the FP8 roofline denominator)
+# ---------------------------------------------------------------------------------------------
+
+PEAKS_FILE = os.path.join(ROOT, "profiles", "tensor_peaks_b200.json")
+
+
+def measure_tensor_peaks(sustain_s: float = 4.0, size: int = 8192) -> dict:
+    """Dense bf16 (torch.matmul) and e4m3 (torch._scaled_mm, bf16 output, fp32
+    tensor scales) GEMMs of size^3: the best of 10 timed launches after warm-up
+    (burst) and the mean over `sustain_s` seconds of back-to-back launches
+    (sustained), with the SM clock sampled by NVML during each."""
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(0)
+    a16 = torch.randn(size, size, device=dev, generator=g).to(torch.bfloat16)
+    b16 = torch.randn(size, size, device=dev, generator=g).to(torch.bfloat16)
+    a8 = a16.to(torch.float8_e4m3fn)
+    b8 = b16.t().contiguous().to(torch.float8_e4m3fn).t()  # column-major second operand
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    flop = 2.0 * size ** 3
+    gemms = {
+        "bf16": lambda: torch.matmul(a16, b16),
+        "fp8_e4m3": lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+    }
+    out = {"gemm": f"{size}x{size}x{size}", "flop_per_launch": flop}
+    for name, fn in gemms.items():
+        for _ in range(20):
+            fn()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            clk.mark()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n, t_end = 0, time.perf_counter() + sustain_s
+            e0.record()
+            while time.perf_counter() < t_end:
+                for _ in range(20):
+                    fn()
+                n += 20
+                torch.cuda.synchronize()
+            e1.record()
+            torch.cuda.synchronize()
+            clk.mark()
+        sus_ms = e0.elapsed_time(e1) / n
+        out[name] = {"burst_tflops": flop / (best * 1e-3) / 1e12,
+                     "sustained_tflops": flop / (sus_ms * 1e-3) / 1e12,
+                     "burst_ms": best, "sustained_ms": sus_ms, "sustained_launches": n,
+                     "clocks_sustained": clk.summary()}
+    out["device"] = torch.cuda.get_device_name()
+    return out
+
+
+def load_fp8_peak(bf16_peak: float, bf16_src: str):
+    """The e4m3 tensor peak: the measured torch._scaled_mm burst figure from the
+    committed peaks file, else the bf16 peak times the nominal e4m3/bf16 ratio."""
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        v = float(d["fp8_e4m3"]["burst_tflops"])
+        return v, (f"measured torch._scaled_mm e4m3 {d['gemm']} burst {v:.1f} TFLOP/s "
+                   f"(profiles/{os.path.basename(PEAKS_FILE)})")
+    except (OSError, ValueError, KeyError, TypeError):
+        return 2.0 * bf16_peak, f"{bf16_src} bf16 burst {bf16_peak} TFLOP/s x2 (nominal fp8/bf16 ratio 4.5/2.25)"
+
+
+# ---------------------------------------------------------------------------------------------
 # reference arm / CPU baseline: the fp64 oracle on a bounded sample of the same workload
 # ---------------------------------------------------------------------------------------------
 
@@ -184,56 +259,87 @@ def workload_desc(w: workloads.Workload) -> str:
             f"seed {w.seed}")
 
 
-def oracle_sample(q, k, v, w: workloads.Workload, target_s: float, max_rows: int | None = None):
-    """Time the fp64 oracle on rows of query head 0 (batch 0), rows spread over the sequence,
-    growing the sample until it has taken about target_s. Returns (TFLOP/s, desc, seconds)."""
+def oracle_heads(q, k, v, w: workloads.Workload, heads) -> float:
+    """Run the fp64 oracle on every row of the given query heads of batch entry 0
+    (each with its own key/value head) and return the seconds it took."""
     import oracle
-    qs = q[0:1, :, 0:1].float().numpy().astype(np.float64)
-    ks = k[0:1, :, 0:1].float().numpy().astype(np.float64)
-    vs = v[0:1, :, 0:1].float().numpy().astype(np.float64)
-    rng = np.random.default_rng(0)
-    n_rows, flops, secs = 64, 0.0, 0.0
-    done_rows = 0
-    while True:
-        rows = np.sort(rng.integers(0, w.N, n_rows))
-        trip = np.stack([np.zeros_like(rows), np.zeros_like(rows), rows], axis=1).astype(np.int64)
+    G = w.Hq // w.Hkv
+    heads = list(heads)
+    kv = [h // G for h in heads]
+    to64 = lambda t: t.float().numpy().astype(np.float64)
+    qs, ks, vs = to64(q[0:1, :, heads]), to64(k[0:1, :, kv]), to64(v[0:1, :, kv])
+    t0 = time.perf_counter()
+    oracle.attention(qs, ks, vs, causal=True)
+    return time.perf_counter() - t0
+
+
+def head_flops(w: workloads.Workload) -> float:
+    """Causal FLOPs of one query head of one batch entry."""
+    return float(w.N) * w.N * (w.d_qk + w.d_v)
+
+
+def cpu_baseline(q, k, v, w: workloads.Workload, full_limit_s: float = 45.0) -> dict:
+    """The oracle, as it stands, on the host cores. One query head is timed first;
+    if the whole workload (every batch entry and head) is then expected to take at
+    most full_limit_s, the whole workload is run and timed in one call."""
+    import oracle
+    t_head = oracle_heads(q, k, v, w, [0])
+    n_heads = w.B * w.Hq
+    cores = len(os.sched_getaffinity(0))
+    if t_head * n_heads <= full_limit_s:
+        to64 = lambda t: t.float().numpy().astype(np.float64)
+        q64, k64, v64 = to64(q), to64(k), to64(v)
         t0 = time.perf_counter()
-        oracle.attention(qs, ks, vs, causal=True, rows=trip)
-        secs += time.perf_counter() - t0
-        flops += float(np.sum(rows + 1)) * 2.0 * (w.d_qk + w.d_v)
-        done_rows += n_rows
-        if secs >= target_s or (max_rows and done_rows >= max_rows):
-            break
-        n_rows = min(n_rows * 2, 1 << 16)
-    desc = (f"{done_rows} query rows of head 0 (batch 0) spread uniformly over N={w.N}, causal, "
-            f"fp64; FLOPs counted as 2*(i+1)*(d_qk+d_v) per row i")
-    return flops / secs / 1e12, desc, secs
+        oracle.attention(q64, k64, v64, causal=True)
+        secs = time.perf_counter() - t0
+        return {"value": w.flops / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"the whole workload ({w.B} x {w.Hq} heads x {w.N} rows), fp64, one call",
+                "seconds": secs}
+    return {"value": head_flops(w) / t_head / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"every row of query head 0 of batch 0 (1/{n_heads} of the workload), fp64",
+            "seconds": t_head}
 
 
 def run_reference(args, rank: int, world: int):
+    """The reference arm: the fp64 oracle on the host cores. A step is every row of
+    one query head (heads taken in turn), a bounded sample of the same workload;
+    ms_per_step is its measured time and value its FLOPs over that time."""
     if rank != 0:
         return
     w = make_workload(args.workload, args.n)
     q, k, v = workloads.draw(w)
     cores = len(os.sched_getaffinity(0))
-    per_step = []
-    desc = ""
+    secs = []
     for i in range(args.warmup + args.steps):
-        tf, desc, secs = oracle_sample(q, k, v, w, target_s=0.5)
+        t = oracle_heads(q, k, v, w, [i % w.Hq])
         if i >= args.warmup:
-            per_step.append(tf)
-    val = statistics.median(per_step)
+            secs.append(t)
+    ms = statistics.mean(secs) * 1e3
+    val = head_flops(w) / (ms * 1e-3) / 1e12
+    desc = (f"one step = every row of one query head of batch 0 (heads in turn; 1/{w.B * w.Hq} of the "
+            f"workload, {head_flops(w):.3e} FLOP), fp64")
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.flops / (val * 1e12) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(w),
-                   "sample": desc,
-                   "ms_per_step": "the whole workload's FLOPs at the sampled rate (each timed step is a sample)"},
+        "config": run_config(args, w, world),
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_config(args, w: workloads.Workload, world: int) -> dict:
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {"workload": workload_desc(w),
+            "step": ("e4m3 quantizer on Q,K,V (per-head scales"
+                     + (", Hadamard on Q,K" if args.hadamard else "") + ") + FP8 attention")
+            if args.dtype == "fp8" else "BF16 attention",
+            "flops_per_step": w.flops, "flop_convention": "B*Hq*N^2*(d_qk+d_v)",
+            "l2": "256 MiB buffer written between timed steps (untimed); inputs exceed L2",
+            "settle": f"{args.settle_s} s of untimed back-to-back steps before timing",
+            "fp8_p": (os.environ.get("B200ATTN_FP8_P") or "lean") if args.dtype == "fp8" else None,
+            "parallelism": f"replicas x{world}"}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -361,6 +467,16 @@ def max_over_ranks(x: float, dist_on: bool, device: str = "cuda") -> float:
     return float(t.item())
 
 
+def kernel_name(dtype: str, w: workloads.Workload) -> str:
+    """The attention kernel (and probability mode) the library runs for this call."""
+    if dtype == "fp8":
+        fp8_p = "mufu" if os.environ.get("B200ATTN_FP8_P") == "mufu" else "lean"
+        kname = "attn_fwd_tile_kernel" if os.environ.get("B200ATTN_FP8_TILE") == "1" else "attn_fwd_kernel"
+        return f"{kname}<{w.d_qk},{w.d_v},fp8,{fp8_p}>"
+    bf16_p = "mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed"
+    return f"attn_fwd_kernel<{w.d_qk},{w.d_v},bf16,{bf16_p}>"
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import bf16_causal_prefill_fwd_b200 as b2
     b2.load_library()
@@ -373,45 +489,56 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peaks, peak_src = load_peaks()
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fp8_peak, fp8_peak_src = load_fp8_peak(bf16_peak, peak_src)
 
-    def measure(dtype, clk=None):
-        path = Path(b2, q, k, v, dtype, args.hadamard)
+    def measure(dtype, wl, tensors, clk=None):
+        path = Path(b2, *tensors, dtype, args.hadamard)
         step_ms, attn_ms = time_path(path, args.steps, args.warmup, args.settle_s, flush, dist_on, clk)
         if b2.check() != 0:
             raise RuntimeError("a kernel reported a timeout")
         ms = max_over_ranks(statistics.mean(step_ms), dist_on)
         ams = max_over_ranks(statistics.mean(attn_ms), dist_on)
-        value = world * w.flops / (ms * 1e-3) / 1e12
-        achieved = w.flops / (ams * 1e-3) / 1e12
-        peak = bf16_peak * (2.0 if dtype == "fp8" else 1.0)
-        fp8_p = os.environ.get("B200ATTN_FP8_P", "lean")
-        kname = "attn_fwd_tile_kernel" if os.environ.get("B200ATTN_FP8_TILE") == "1" else "attn_fwd_kernel"
-        bf16_p = "mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed"
-        kernel_key = (f"{kname}<{w.d_qk},{w.d_v},fp8,{'mufu' if fp8_p == 'mufu' else 'lean'}>"
-                      if dtype == "fp8" else f"attn_fwd_kernel<{w.d_qk},{w.d_v},bf16,{bf16_p}>")
+        value = world * wl.flops / (ms * 1e-3) / 1e12
+        achieved = wl.flops / (ams * 1e-3) / 1e12
+        peak = fp8_peak if dtype == "fp8" else bf16_peak
+        kernel_key = kernel_name(dtype, wl)
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic_for(kernel_key, w.name),
+                "frac": achieved / peak, "traffic": traffic_for(kernel_key, wl.name),
                 "kernel": kernel_key, "kernel_ms": ams,
-                "peak_source": (f"{peak_src} bf16 burst {bf16_peak} TFLOP/s"
-                                + (" x2 (nominal fp8/bf16 ratio 4.5/2.25)" if dtype == "fp8" else "")),
+                "peak_source": fp8_peak_src if dtype == "fp8" else f"{peak_src} bf16 burst {bf16_peak} TFLOP/s",
                 "frac_of_spec_dense": achieved / (4500.0 if dtype == "fp8" else 2250.0)}
         quant = None
         if dtype == "fp8":
             qms = max_over_ranks(statistics.mean([s - a for s, a in zip(step_ms, attn_ms)]), dist_on)
-            quant = quantizer_summary(qms, w, hbm_peak)
+            quant = quantizer_summary(qms, wl, hbm_peak)
         return {"value": value, "ms_per_step": ms, "roofline": roof, "quantizer": quant,
                 "launches": path.launches_per_step * args.steps,
                 "step_ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))]}
 
     with ClockSampler(local_rank) as clk:
-        main = measure(args.dtype, clk)
+        main = measure(args.dtype, w, (q, k, v), clk)
     clocks = clk.summary()
     energy = measure_energy(clk, Path(b2, q, k, v, args.dtype, args.hadamard), w.flops, args.energy_s)
     other = None
     if not args.no_other_dtype:
         other_dtype = "bf16" if args.dtype == "fp8" else "fp8"
-        other = measure(other_dtype)
+        with ClockSampler(local_rank) as clk_o:
+            other = measure(other_dtype, w, (q, k, v), clk_o)
         other["dtype"] = other_dtype
+        other["clocks"] = clk_o.summary()
+
+    # The spec point: the Gaussian sweep's N = 32768 (B = 1) layer, both dtypes.
+    at_32k = None
+    if not args.no_at_32k and w.name != "sweep32768":
+        w32 = workloads.sweep(32768)
+        t32 = tuple(t.cuda() for t in workloads.draw(w32))
+        at_32k = {"workload": workload_desc(w32), "flops_per_step": w32.flops}
+        for dt in ("fp8", "bf16"):
+            with ClockSampler(local_rank) as clk32:
+                r = measure(dt, w32, t32, clk32)
+            at_32k[dt] = {"value": r["value"], "ms_per_step": r["ms_per_step"], "roofline": r["roofline"],
+                          "quantizer": r["quantizer"], "clocks": clk32.summary()}
+        del t32
 
     e2e = None
     if not args.no_e2e:
@@ -419,27 +546,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
-        tf, desc, secs = oracle_sample(q_cpu, k_cpu, v_cpu, w, target_s=10.0)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-               "sample": desc, "seconds": secs}
+        cpu = cpu_baseline(q_cpu, k_cpu, v_cpu, w)
 
     if rank == 0:
+        config = run_config(args, w, world)
         line = {
             "metric": METRIC, "value": main["value"], "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp8_e4m3" if args.dtype == "fp8" else "bf16", "data": "synthetic",
-            "config": {"workload": workload_desc(w),
-                       "step": ("e4m3 quantizer on Q,K,V (per-head scales"
-                                + (", Hadamard on Q,K" if args.hadamard else "") + ") + FP8 attention")
-                       if args.dtype == "fp8" else "BF16 attention",
-                       "flops_per_step": w.flops, "flop_convention": "B*Hq*N^2*(d_qk+d_v)",
-                       "l2": "256 MiB buffer written between timed steps (untimed); inputs exceed L2",
-                       "settle": f"{args.settle_s} s of untimed back-to-back steps before timing",
-                       "fp8_p": os.environ.get("B200ATTN_FP8_P", "lean") if args.dtype == "fp8" else None,
-                       "bf16_p": (("mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed")
-                                  if args.dtype == "bf16" else None),
-                       "parallelism": f"replicas x{world}"},
+            "config": config,
             "roofline": main["roofline"],
             "quantizer": main["quantizer"],
             "clocks": clocks,
@@ -451,6 +567,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         }
         if other is not None:
             line["other_dtype"] = other
+        if at_32k is not None:
+            line["at_32k"] = at_32k
         print(json.dumps(line), flush=True)
 
 
@@ -501,6 +619,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.measure_peaks:
+        torch.cuda.set_device(local_rank)
+        print(json.dumps(measure_tensor_peaks()), flush=True)
         return
     dist_on = world > 1
     if dist_on:

@@ -90,6 +90,12 @@ namespace b200 {
 constexpr int kBM = 128;         // query rows per tile
 constexpr int kBN = 128;         // keys per block
 constexpr int kAttnThreads = 384;
+// Registers per thread: at launch (65536 / 384 rounded down to a multiple of 8),
+// then after the role split (warps 0-3 give registers up, warps 4-11 take them).
+constexpr int kRegsAtLaunch = 168;
+constexpr int kRegsLow = 72;
+constexpr int kRegsHigh = 208;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kAttnThreads * kRegsAtLaunch, "register split");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 constexpr int kStatusTimeout = -4;                 // B200ATTN_ERR_TIMEOUT
 
@@ -347,6 +353,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp < 4) {
+    // Register split between roles: the producer and issuer warps need few
+    // registers, the softmax warps hold a 128-entry score row each. The block
+    // is launched with kRegsAtLaunch per thread (the host checks), and
+    // 128 * kRegsLow + 256 * kRegsHigh does not exceed 384 * kRegsAtLaunch.
+    setmaxnreg_dec<kRegsLow>();
   if (warp == 0 || warp == 3) {
     // ------------------------------------------------------------ TMA producers
     // warp 0: Q tiles and K blocks; warp 3: V blocks. Each walks the same unit
@@ -398,7 +410,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) __nanosleep(200000);  // let copies already in flight land before the CTA exits
     }
     __syncwarp();
-  } else if (warp == 1 || warp == 2) {
+  } else {
     // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
       // Descriptor low words of every buffer, computed once; an MMA along K adds
@@ -559,7 +571,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsHigh>();
     // ------------------------------------------------------------ softmax + epilogue
     const int t = (warp - 4) >> 2;            // query tile of this warpgroup
     const int r = threadIdx.x - 128 - 128 * t;  // row within the tile == TMEM lane

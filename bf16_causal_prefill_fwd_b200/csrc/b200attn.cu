@@ -88,6 +88,20 @@ int device_ok(int* sm_count) {
   return B200ATTN_OK;
 }
 
+// True if the kernel was built with exactly R registers per thread (cached per kernel).
+template <int R>
+bool regs_match(const void* kern) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, bool>> seen;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& e : seen)
+    if (e.first == kern) return e.second;
+  cudaFuncAttributes a;
+  const bool ok = cudaFuncGetAttributes(&a, kern) == cudaSuccess && a.numRegs == R;
+  seen.emplace_back(kern, ok);
+  return ok;
+}
+
 template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S>
 int launch_attn_t(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
@@ -99,6 +113,10 @@ int launch_attn_t(const void* q, const void* k, const void* v, const AttnParams&
   auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, FMA_P, SHARED_S>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
+  // The kernel's role split (setmaxnreg) hands out registers from the block's
+  // launch allocation; a build with fewer registers per thread than it assumes
+  // would leave the softmax warps waiting for registers that do not exist.
+  if (!regs_match<b200::kRegsAtLaunch>(reinterpret_cast<const void*>(kern))) return B200ATTN_ERR_UNSUPPORTED;
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
   kern<<<grid, b200::kAttnThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;

@@ -243,7 +243,10 @@ int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v,
  *   rejected with B200ATTN_ERR_WORKSPACE before anything is launched.
  * - The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture.
+ *   first call before any stream capture. The cached address belongs to the
+ *   device's context at that time: after cudaDeviceReset (or anything else
+ *   that destroys the primary context) this entry point must not be called
+ *   again in the same process.
  * - Every call on a device shares the one array, which keeps the last call's
  *   partial absmax values (each call overwrites the slots it reads, so nothing
  *   needs clearing). Calls that overlap on the GPU (on different streams, or

@@ -69,3 +69,17 @@ def gather_sample(o_gpu, heads, rows):
     idx_r = torch.tensor(rows, device=o_gpu.device)
     sel = o_gpu[0].index_select(0, idx_r).index_select(1, idx_h)   # [rows, heads, d]
     return sel.permute(1, 0, 2).double().cpu().numpy()
+
+
+def error_report(got: np.ndarray, ref: np.ndarray) -> dict:
+    """Errors of a sampled output [heads, rows, d] against the fp64 oracle: the
+    relative RMS over the whole sample (the gated figure), the largest per-head
+    relative RMS, and the largest absolute element error."""
+    per_head = [oracle.rel_rms(got[h], ref[h]) for h in range(got.shape[0])]
+    return {"rel_rms": oracle.rel_rms(got, ref), "max_head_rel_rms": max(per_head),
+            "max_abs": float(np.max(np.abs(got - ref)))}
+
+
+def fmt_errors(e: dict) -> str:
+    return (f"rel-rms {e['rel_rms']:.2e} (worst head {e['max_head_rel_rms']:.2e}, "
+            f"max-abs {e['max_abs']:.2e})")

@@ -3,6 +3,7 @@ gets the slowest rank's time, and the reference arm runs on rank 0 only. Also th
 quantizer's HBM-roofline arithmetic."""
 import os
 import socket
+import time
 
 import pytest
 import torch
@@ -43,12 +44,14 @@ def test_max_over_ranks_with_gloo():
         assert dict(results) == {0: 2.5, 1: 2.5}
 
 
+class RefArgs:
+    workload, n, warmup, steps, dtype, hadamard, settle_s = "tiny", None, 3, 1, "fp8", False, 1.0
+
+
 def test_reference_arm_other_ranks_do_no_work(capsys):
     import bench
 
-    class A:
-        workload, n, warmup, steps = "tiny", None, 3, 1
-    bench.run_reference(A(), rank=1, world=2)
+    bench.run_reference(RefArgs(), rank=1, world=2)
     assert capsys.readouterr().out == ""
 
 
@@ -73,10 +76,14 @@ def test_reference_arm_line_on_rank_zero(capsys):
     import json
     import bench
 
-    class A:
-        workload, n, warmup, steps = "tiny", None, 3, 1
-    bench.run_reference(A(), rank=0, world=1)
+    t0 = time.perf_counter()
+    bench.run_reference(RefArgs(), rank=0, world=1)
+    wall_ms = (time.perf_counter() - t0) * 1e3
     line = json.loads(capsys.readouterr().out.strip())
+    # a step is a measured sample (one query head), so the timed steps fit in the run
+    assert 0 < line["ms_per_step"] * line["steps"] <= wall_ms
+    w = bench.make_workload("tiny", None)
+    assert line["config"] == bench.run_config(RefArgs(), w, 1)
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC
     assert line["value"] > 0 and line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
     assert line["config"]["workload"] == bench.workload_desc(bench.make_workload("tiny", None))

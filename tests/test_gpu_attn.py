@@ -12,7 +12,8 @@ import torch
 import oracle
 import workloads
 import bf16_causal_prefill_fwd_b200 as b2
-from helpers import (BF16_TOL, FP8_TOL, f32, gather_sample, oracle_fp8_inputs, oracle_on_sample, subset_problem,
+from helpers import (BF16_TOL, FP8_TOL, error_report, f32, fmt_errors, gather_sample, oracle_fp8_inputs,
+                     oracle_on_sample, subset_problem,
                      sampled_rows, to_gpu_fp8)
 
 pytestmark = pytest.mark.gpu
@@ -300,36 +301,49 @@ def test_bitwise_deterministic_over_1000_launches(dtype, monkeypatch):
 
 
 # ---------------------------------------------------------------- full-size workloads, sampled rows
+#
+# Each case prints, next to the gated relative RMS, the worst per-head relative
+# RMS and the largest absolute error of the sample; the per-head figure is gated
+# at the same tolerance.
 
 FULL = {
     "gqa7b": workloads.gqa7b,
     "qknorm": workloads.qknorm,
     "mla": workloads.mla,
+    "mla32k": lambda: workloads.mla(32768),
+    "sweep32k": lambda: workloads.sweep(32768),
 }
 
 
-@pytest.mark.parametrize("name", ["gqa7b", "mla"])
+def sample_of(w):
+    return sorted({0, 1, w.Hq // w.Hkv, w.Hq - 1}), sampled_rows(w.N)
+
+
+def assert_within(e, tol):
+    assert e["rel_rms"] <= tol, e
+    assert e["max_head_rel_rms"] <= tol, e
+
+
+@pytest.mark.parametrize("name", ["gqa7b", "qknorm", "mla", "mla32k", "sweep32k"])
 def test_full_size_bf16_sampled(name):
     w = FULL[name]()
     q, k, v = workloads.draw(w)
     o, _ = run_bf16(q, k, v)
-    heads = sorted({0, 1, w.Hq // w.Hkv, w.Hq - 1})
-    rows = sampled_rows(w.N)
+    heads, rows = sample_of(w)
     ref, _ = oracle_on_sample(q, k, v, heads, rows)
-    err = oracle.rel_rms(gather_sample(o, heads, rows), ref)
-    print(f"{name} bf16 sampled rel-rms {err:.2e}")
-    assert err <= BF16_TOL
+    e = error_report(gather_sample(o, heads, rows), ref)
+    print(f"{name} N={w.N} bf16 sampled {fmt_errors(e)}")
+    assert_within(e, BF16_TOL)
     assert torch.isfinite(o.float()).all()
 
 
 @pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("gqa7b", True), ("qknorm", False), ("qknorm", True),
-                                           ("mla", False)])
+                                           ("mla", False), ("mla32k", False)])
 def test_full_size_fp8_sampled(name, hadamard, monkeypatch):
     """Both ways of forming P, on the oracle's codes of the full layer; rows sampled."""
     w = FULL[name]()
     q, k, v = workloads.draw(w)
-    heads = sorted({0, 1, w.Hq // w.Hkv, w.Hq - 1})
-    rows = sampled_rows(w.N)
+    heads, rows = sample_of(w)
     codes, deq = oracle_fp8_inputs(q, k, v, hadamard=hadamard)
     ref8, _ = oracle_on_sample(*deq, heads, rows)
     ref, _ = oracle_on_sample(q, k, v, heads, rows)
@@ -337,15 +351,70 @@ def test_full_size_fp8_sampled(name, hadamard, monkeypatch):
         monkeypatch.setenv("B200ATTN_FP8_P", mode)
         o, _ = run_fp8(codes)
         got = gather_sample(o, heads, rows)
-        err = oracle.rel_rms(got, ref8)
-        print(f"{name} fp8[{mode}] (hadamard={hadamard}) rel-rms {err:.2e}; "
+        e = error_report(got, ref8)
+        print(f"{name} N={w.N} fp8[{mode}] (hadamard={hadamard}) {fmt_errors(e)}; "
               f"vs unquantised fp64 {oracle.rel_rms(got, ref):.2e}")
-        assert err <= FP8_TOL
+        assert_within(e, FP8_TOL)
 
 
-# ---------------------------------------------------------------- sequence sweep, FP8 error at each N
+@pytest.mark.parametrize("fp8_kernel", ["tile"], indirect=True)
+@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
+def test_full_size_fp8_tile_kernel_sampled(fp8_p, fp8_kernel):
+    """The one-tile FP8 kernel on the full 7B-style layer (N = 16384), where its
+    K/V rings wrap many times per unit."""
+    w = workloads.gqa7b()
+    q, k, v = workloads.draw(w)
+    heads, rows = sample_of(w)
+    codes, deq = oracle_fp8_inputs(q, k, v)
+    ref8, _ = oracle_on_sample(*deq, heads, rows)
+    o, _ = run_fp8(codes)
+    e = error_report(gather_sample(o, heads, rows), ref8)
+    print(f"gqa7b fp8[{fp8_p}, one-tile kernel] {fmt_errors(e)}")
+    assert_within(e, FP8_TOL)
 
-@pytest.mark.parametrize("N", [1024, 2048, 4096, 8192, 16384, 32768])
+
+@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
+def test_full_size_fp8_per_block_scales_sampled(fp8_p):
+    """Scales per (b, h, 128-token block) on the full 7B-style layer (N = 16384):
+    128 scale blocks per head, so the kernel's V reference scale is raised and O
+    rescaled many times along each row."""
+    w = workloads.gqa7b()
+    q, k, v = workloads.draw(w)
+    heads, rows = sample_of(w)
+    codes, deq = oracle_fp8_inputs(q, k, v, granularity="block")
+    ref8, _ = oracle_on_sample(*deq, heads, rows)
+    q8, sq, k8, sk, v8, sv = to_gpu_fp8(codes)
+    o = b2.attn_fwd(q8, k8, v8, q_scale=sq, k_scale=sk, v_scale=sv, scale_granularity="block")
+    assert b2.check() == 0
+    e = error_report(gather_sample(o, heads, rows), ref8)
+    print(f"gqa7b fp8[{fp8_p}, per-block scales] {fmt_errors(e)}")
+    assert_within(e, FP8_TOL)
+
+
+# ---------------------------------------------------------------- sequence sweep, error at each N
+
+SWEEP_N = [1024, 2048, 4096, 8192, 16384, 32768]
+
+
+@pytest.mark.parametrize("N", SWEEP_N)
+def test_sweep_bf16_error_sampled(N):
+    """The Gaussian sweep (B = 32768/N) in BF16: sampled rows of the first and
+    last query head of the first and last batch entry against fp64."""
+    w = workloads.sweep(N)
+    q, k, v = workloads.draw(w)
+    o, _ = run_bf16(q, k, v)
+    heads, rows = [0, w.Hq - 1], sampled_rows(N)
+    errs = []
+    for b in sorted({0, w.B - 1}):
+        qs, ks, vs = q[b:b + 1], k[b:b + 1], v[b:b + 1]
+        ref, _ = oracle_on_sample(qs, ks, vs, heads, rows)
+        errs.append(error_report(gather_sample(o[b:b + 1], heads, rows), ref))
+    for b, e in zip(sorted({0, w.B - 1}), errs):
+        print(f"sweep N={N} B={w.B} batch {b} bf16 {fmt_errors(e)}")
+        assert_within(e, BF16_TOL)
+
+
+@pytest.mark.parametrize("N", SWEEP_N)
 def test_sweep_fp8_error_sampled(N):
     """The Gaussian sweep (B = 32768/N) through the product path: Q, K, V
     quantised on the GPU, FP8 attention. The oracle quantises the sampled heads
@@ -371,6 +440,6 @@ def test_sweep_fp8_error_sampled(N):
     ref8, _ = oracle_on_sample(*deq, sub, rows)
     ref, _ = oracle_on_sample(qs, ks, vs, sub, rows)
     got = gather_sample(o, heads, rows)
-    err, err_unq = oracle.rel_rms(got, ref8), oracle.rel_rms(got, ref)
-    print(f"sweep N={N} B={w.B} fp8 rel-rms {err:.2e}; vs unquantised fp64 {err_unq:.2e}")
-    assert err <= FP8_TOL, err
+    e = error_report(got, ref8)
+    print(f"sweep N={N} B={w.B} fp8 {fmt_errors(e)}; vs unquantised fp64 {oracle.rel_rms(got, ref):.2e}")
+    assert_within(e, FP8_TOL)

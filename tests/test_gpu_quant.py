@@ -44,7 +44,10 @@ def test_zero_and_saturation_cases():
 
 
 @pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("qknorm", True)])
-def test_full_size_q_bit_exact(name, hadamard):
+def test_full_size_single_tensor_bit_exact(name, hadamard):
+    """The one-tensor quantizer on the full layer: K and V in full, and Q on
+    four of its 32 heads (per-head scales depend on that head's values only, so
+    the oracle quantises the head subset on its own)."""
     w = workloads.BY_NAME[name]()
     q, k, v = workloads.draw(w)
     for t, rot in ((k, hadamard), (v, False)):
@@ -52,6 +55,11 @@ def test_full_size_q_bit_exact(name, hadamard):
         ref_codes, ref_scale = oracle.quantize_fp8(f32(t), "head", rot)
         assert np.array_equal(scale, ref_scale)
         assert np.array_equal(codes, ref_codes)
+    heads = [0, 1, w.Hq // 2, w.Hq - 1]
+    codes, scale = gpu_quant(q, "head", hadamard)
+    ref_codes, ref_scale = oracle.quantize_fp8(f32(q[:, :, heads].contiguous()), "head", hadamard)
+    assert np.array_equal(scale[:, heads], ref_scale)
+    assert np.array_equal(codes[:, :, heads], ref_codes)
 
 
 # (2, 4000, 8, 2, 128) has more 128-token head blocks (768) than the persistent

@@ -63,3 +63,21 @@ def test_static_scratch_quantizer_rejects_problems_beyond_its_capacity():
     n_over = (CAPACITY + 1) * 128
     assert lib.b200attn_quantize_fp8_static(fake, fake, fake, 1, n_over, 1, 128, 0, None) == -5
     assert lib.b200attn_quantize_fp8_static(fake, fake, fake, 2, CAPACITY // 2 * 128, 2, 128, 0, None) == -5
+
+
+def test_static_scratch_quantizer_at_exactly_its_capacity():
+    """A problem that fills every slot of the static scratch (B*H*ceil(N/128) ==
+    65536: 16 heads of 524288 tokens, 2 GiB of bf16) matches the workspace
+    quantizer; one 128-token block more is rejected before anything runs."""
+    lib = lib_with_static()
+    B, H, d = 1, 16, 128
+    N = CAPACITY // H * 128
+    g = torch.Generator(device="cuda").manual_seed(12)
+    x = (torch.randn(B, N, H, d, device="cuda", generator=g) * 4).to(torch.bfloat16)
+    codes, scale, ref_codes, ref_scale = quantize_both(lib, x, False)
+    assert torch.equal(scale, ref_scale)
+    assert torch.equal(codes, ref_codes)
+    del codes, ref_codes
+    rc = lib.b200attn_quantize_fp8_static(x.data_ptr(), x.data_ptr(), scale.data_ptr(), B, N + 1, H, d, 0,
+                                          torch.cuda.current_stream().cuda_stream)
+    assert rc == -5
