@@ -88,7 +88,7 @@ def load_peaks():
 
 def kernel_sources_sha() -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd_kernel.cuh", "attn_fwd_tile_kernel.cuh", "sm100_ptx.cuh"):
+    for f in ("attn_fwd_kernel.cuh", "attn_fwd_pair_kernel.cuh", "attn_fwd_tile_kernel.cuh", "sm100_ptx.cuh"):
         with open(os.path.join(ROOT, "bf16_causal_prefill_fwd_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -471,7 +471,12 @@ def kernel_name(dtype: str, w: workloads.Workload) -> str:
     """The attention kernel (and probability mode) the library runs for this call."""
     if dtype == "fp8":
         fp8_p = "mufu" if os.environ.get("B200ATTN_FP8_P") == "mufu" else "lean"
-        kname = "attn_fwd_tile_kernel" if os.environ.get("B200ATTN_FP8_TILE") == "1" else "attn_fwd_kernel"
+        if os.environ.get("B200ATTN_FP8_TILE") == "1":
+            kname = "attn_fwd_tile_kernel"
+        elif os.environ.get("B200ATTN_FP8_PAIR") == "1":
+            kname = "attn_fwd_pair_kernel"
+        else:
+            kname = "attn_fwd_kernel"
         return f"{kname}<{w.d_qk},{w.d_v},fp8,{fp8_p}>"
     bf16_p = "mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed"
     return f"attn_fwd_kernel<{w.d_qk},{w.d_v},bf16,{bf16_p}>"

@@ -66,6 +66,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.b200attn_version.argtypes = []
     lib.b200attn_selftest_wait_timeout.restype = i
     lib.b200attn_selftest_wait_timeout.argtypes = [i, vp]
+    lib.b200attn_trace_read.restype = i
+    lib.b200attn_trace_read.argtypes = [vp, i, i, i]
     _lib = lib
     return lib
 

@@ -1,6 +1,6 @@
 """Build libb200attn.so in-tree with nvcc for sm_100a.
 
-    python -m bf16_causal_prefill_fwd_b200.build [--force] [--verbose]
+    python -m bf16_causal_prefill_fwd_b200.build [--force] [--verbose] [--trace]
 
 The library is a single translation unit (csrc/b200attn.cu) with the CUDA
 runtime linked statically, so it loads next to any PyTorch build.
@@ -19,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libb200attn.so")
+TRACE_LIB_PATH = os.path.join(LIB_DIR, "libb200attn_trace.so")  # same library with -DATTN_TRACE
 HEADER = os.path.join(ROOT, "include", "b200attn.h")
 
 NVCC_FLAGS = [
@@ -40,35 +41,41 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) + [HEADER])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+def up_to_date(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB_PATH
+def build(force: bool = False, verbose: bool = False, trace: bool = False) -> str:
+    """Build lib/libb200attn.so, or with trace=True lib/libb200attn_trace.so (the
+    kernels record per-block events for b200attn_trace_read)."""
+    path = TRACE_LIB_PATH if trace else LIB_PATH
+    if not force and up_to_date(path):
+        return path
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
+    tmp = path + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *NVCC_FLAGS]
+    if trace:
+        cmd += ["-DATTN_TRACE"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += ["-o", tmp, os.path.join(CSRC, "b200attn.cu")]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libb200attn.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(path)}")
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--trace", action="store_true", help="build lib/libb200attn_trace.so (-DATTN_TRACE)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, trace=a.trace))

@@ -83,6 +83,7 @@
 
 #include <cuda_bf16.h>
 
+#include "attn_trace.cuh"
 #include "sm100_ptx.cuh"
 
 namespace b200 {
@@ -308,6 +309,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  trace_begin();
+  if (threadIdx.x == 0) trace(kEvLaunch, gridDim.x);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -400,6 +403,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (it >= static_cast<uint32_t>(nslot) && !(ok = mbar_wait(bEmpty + 8 * s, ((it / nslot) - 1) & 1, abort_flag)))
             break;
           const uint32_t bar = bFull + 8 * s;
+          trace(is_k ? kEvKLoad : kEvVLoad, it);
           mbar_arrive_expect_tx(bar, slot_bytes);
           for (int c = 0; c < chunks; ++c)
             tma_load_4d_hint(ring + s * slot_bytes + c * C::CHUNK_BYTES, tm, bar, c * C::CHUNK_ELEMS, x.hkv,
@@ -474,6 +478,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int n_t = t ? x.n1 : x.n0;
                 if (j >= n_t) continue;
                 if (nq > 0 && !(ok = mbar_wait(bSFree, (nq - 1) & 1, abort_flag))) break;
+                trace(kEvQkIssue, nq);
                 ++nq;
                 tc_fence_after();
                 issue_qk(t, s);
@@ -498,6 +503,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   oe_par[t] ^= 1;
                 }
                 if (!ok) break;
+                trace(kEvPvIssue, g);
                 tc_fence_after();
                 issue_pv(t, t * C::PB + pb, s, j > 0);
                 tc_commit(bPDone + 8 * (t * C::PBX + pb));
@@ -585,6 +591,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t bOf = bOFull + 8 * t, bOe = bOEmpty + 8 * t;
     uint32_t s_par = 0, o_par = 0;
     uint32_t g = 0;  // key blocks this warpgroup has finished (SS buffer and parity index)
+    const bool tracer = (warp & 3) == 0 && lane == 0;  // one thread per softmax warpgroup logs events
     bool ok = true;
 
     for (int k = 0; ok; ++k) {
@@ -620,6 +627,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool mma_sum = C::RS && !p.per_block;
 
       for (int i = 0; i < n_t; ++i, ++g) {
+        if (tracer) trace(kEvSoftmaxWaitS, g);
         ok = __all_sync(0xffffffffu, mbar_wait(bS, s_par, abort_flag));
         if (!ok) break;
         s_par ^= 1;
@@ -638,6 +646,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_fence_before();
           mbar_arrive(bSFree);  // S may take the next product now
         }
+        if (tracer) trace(kEvSoftmaxHaveS, g);
 
         const int kv0 = i * kBN;
         if (p.causal) {
@@ -690,6 +699,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_run = m_new;
         }
         l_run *= alpha;
+        if (tracer) trace(kEvSoftmaxMaxDone, g);
         const bool need = need_m || v_alpha != 1.0f;
         alpha *= v_alpha;
 
@@ -854,6 +864,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bPFull + 8 * (t * C::PBX + g % C::PBX));
+        if (tracer) trace(kEvSoftmaxPDone, g);
       }
       if (!ok) break;
 
@@ -893,6 +904,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             (m_run + __log2f(l_run) - C::E_SHIFT) * 0.6931471805599453f;
       tc_fence_before();
       mbar_arrive(bOe);
+      if (tracer) trace(kEvEpilogue, g);
     }
   }
 
@@ -904,6 +916,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  trace_end();
 }
 
 // Failure-path self-test: one thread waits, through the same bounded wait as

@@ -15,6 +15,7 @@
 
 #include "../../include/b200attn.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_fwd_pair_kernel.cuh"
 #include "attn_fwd_tile_kernel.cuh"
 #include "quant_kernel.cuh"
 
@@ -54,6 +55,24 @@ bool make_tmap(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, int N, i
                          const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The same map with another box and swizzle: box = {box_inner elements of d, 1
+// head, box_rows tokens, 1}; swizzle_bytes 64 or 128.
+bool make_tmap_box(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, int N, int B, int box_inner,
+                   int box_rows, int swizzle_bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t esz = fp8 ? 1 : 2;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * esz, (cuuint64_t)H * d * esz, (cuuint64_t)N * H * d * esz};
+  const cuuint32_t box[4] = {(cuuint32_t)box_inner, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                         const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -154,6 +173,53 @@ int launch_attn_tile(const void* q, const void* k, const void* v, AttnParams p, 
   const int grid = p.n_units < sm_count ? p.n_units : sm_count;
   kern<<<grid, b200::kAttnThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+// FP8 with per-head scales on CTA pairs (attn_fwd_pair_kernel): one query tile
+// per SM, the two tiles of a unit on the two SMs of a cluster.
+template <int DQK, int DV, bool FMA_P>
+int launch_attn_pair(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v,
+                     cudaStream_t stream) {
+  using C = b200::PairCfg<DQK, DV, FMA_P>;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_box(&tq, q, true, d_qk, p.Hq, p.N, p.B, 128, 128, 128) ||
+      !make_tmap_box(&tk, k, true, d_qk, p.Hkv, p.N, p.B, 128, 64, 128) ||
+      !make_tmap_box(&tv, v, true, d_v, p.Hkv, p.N, p.B, 64, 128, 64))
+    return B200ATTN_ERR_CUDA;
+  auto kern = b200::attn_fwd_pair_kernel<DQK, DV, FMA_P>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return B200ATTN_ERR_CUDA;
+  if (!regs_match<b200::kRegsAtLaunch>(reinterpret_cast<const void*>(kern))) return B200ATTN_ERR_UNSUPPORTED;
+  // Clusters that can be resident at once (a persistent grid larger than that
+  // would leave clusters waiting for others to finish), looked up once per device.
+  static std::mutex mu;
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return B200ATTN_ERR_CUDA;
+  int max_clusters = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2, 1, 1);
+      cfg.blockDim = dim3(b200::kAttnThreads, 1, 1);
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return B200ATTN_ERR_CUDA;
+      cached[dev] = n;
+    }
+    max_clusters = cached[dev];
+  }
+  const int clusters = p.n_units < max_clusters ? p.n_units : max_clusters;
+  kern<<<2 * clusters, b200::kAttnThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+// FP8 per-head kernel on CTA pairs (B200ATTN_FP8_PAIR=1) or the two-tile
+// kernel on one SM (default); read on every call so A/B runs need no rebuild.
+bool fp8_pair_kernel() {
+  const char* e = std::getenv("B200ATTN_FP8_PAIR");
+  return e && std::strcmp(e, "1") == 0;
 }
 
 // Which FP8 per-head kernel runs: the two-tile kernel (default, faster on the
@@ -296,6 +362,14 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
     }
     if (d_qk == 128) return launch_attn_tile<128, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn_tile<192, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
+  }
+  if (!p.per_block && fp8_pair_kernel()) {
+    if (fp8_lean_p()) {
+      if (d_qk == 128) return launch_attn_pair<128, 128, true>(q, k, v, p, d_qk, d_v, st);
+      return launch_attn_pair<192, 128, true>(q, k, v, p, d_qk, d_v, st);
+    }
+    if (d_qk == 128) return launch_attn_pair<128, 128, false>(q, k, v, p, d_qk, d_v, st);
+    return launch_attn_pair<192, 128, false>(q, k, v, p, d_qk, d_v, st);
   }
   if (fp8_lean_p()) {
     if (d_qk == 128) return launch_attn<128, 128, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
@@ -543,6 +617,36 @@ int b200attn_selftest_wait_timeout(int limit_us, void* stream) {
   b200::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(limit_us) * 1000ull);
   return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+int b200attn_trace_read(void* out, int cta, int cap, int reset) {
+#ifdef ATTN_TRACE
+  if (cta < 0 || cta >= b200::kTraceCtas || cap < 0 || (cap > 0 && !out)) return B200ATTN_ERR_INVALID;
+  if (cudaDeviceSynchronize() != cudaSuccess) return B200ATTN_ERR_CUDA;
+  uint32_t n[b200::kTraceWarps] = {};
+  if (cudaMemcpyFromSymbol(n, b200::g_attn_trace_n, sizeof(n), sizeof(n) * cta) != cudaSuccess)
+    return B200ATTN_ERR_CUDA;
+  int m = 0;
+  for (int w = 0; w < b200::kTraceWarps && m < cap; ++w) {
+    const int nw = std::min<int>(std::min<uint32_t>(n[w], b200::kTracePerWarp), cap - m);
+    const size_t off = sizeof(b200::TraceRec) * (static_cast<size_t>(cta) * b200::kTraceWarps + w) * b200::kTracePerWarp;
+    if (nw > 0 && cudaMemcpyFromSymbol(static_cast<b200::TraceRec*>(out) + m, b200::g_attn_trace,
+                                       sizeof(b200::TraceRec) * nw, off) != cudaSuccess)
+      return B200ATTN_ERR_CUDA;
+    m += nw;
+  }
+  if (reset) {
+    static const uint32_t zero[b200::kTraceCtas][b200::kTraceWarps] = {};
+    if (cudaMemcpyToSymbol(b200::g_attn_trace_n, zero, sizeof(zero)) != cudaSuccess) return B200ATTN_ERR_CUDA;
+  }
+  return m;
+#else
+  (void)out;
+  (void)cta;
+  (void)cap;
+  (void)reset;
+  return B200ATTN_ERR_UNSUPPORTED;
+#endif
 }
 
 int b200attn_check(void* stream) {

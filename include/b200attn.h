@@ -276,6 +276,27 @@ int b200attn_check(void* stream);
  */
 int b200attn_selftest_wait_timeout(int limit_us, void* stream);
 
+/*
+ * b200attn_trace_read -- per-block event trace of the attention kernels, for
+ * profiling the pipeline (which role waits for which). Only a library built
+ * with tracing (python -m bf16_causal_prefill_fwd_b200.build --trace, file
+ * lib/libb200attn_trace.so) records anything; the normal library returns
+ * B200ATTN_ERR_UNSUPPORTED. The pages have no counterpart: they show a thread
+ * trace of their own kernel ("ZYFA 如何工作？", 双波乒乓调度), and this is the
+ * tool that gives the same view of this library's kernels.
+ *
+ * The traced build records, for the first 4 CTAs of each launch, up to 4096
+ * events per warp: {uint32 event | warp << 8, uint32 block counter, uint64
+ * clock64 of the SM}, 16 bytes each (event ids in csrc/attn_trace.cuh); a
+ * launch overwrites the previous one's records.
+ * out    host buffer of cap records (may be NULL when cap == 0)
+ * cta    0 .. 3
+ * reset  nonzero: clear every CTA's record count afterwards
+ * Synchronises the device. Returns the number of records copied (>= 0), or
+ * INVALID, UNSUPPORTED, CUDA.
+ */
+int b200attn_trace_read(void* out, int cta, int cap, int reset);
+
 /* Static description of a status code; never NULL. */
 const char* b200attn_strerror(int code);
 

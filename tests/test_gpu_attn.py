@@ -58,21 +58,26 @@ SMALL = [
 FP8_P = ["lean", "mufu"]
 
 
-# FP8 with per-head scales has two kernels: two query tiles per CTA (default)
-# and one tile per CTA (B200ATTN_FP8_TILE=1); the tests marked with this
-# fixture run both.
-FP8_KERNELS = ["pair", "tile"]
+# FP8 with per-head scales has three kernels: both query tiles of a unit on one
+# SM (default), the two tiles on the two SMs of a CTA pair
+# (B200ATTN_FP8_PAIR=1), and one tile per unit on one SM (B200ATTN_FP8_TILE=1);
+# the tests marked with this fixture run all three.
+FP8_KERNELS = ["pair", "two", "tile"]
+FP8_KERNEL_ENV = {"pair": ("0", "1"), "two": ("0", "0"), "tile": ("1", "1")}  # (FP8_TILE, FP8_PAIR)
 
 
 @pytest.fixture
 def fp8_kernel(request):
-    old = os.environ.get("B200ATTN_FP8_TILE")
-    os.environ["B200ATTN_FP8_TILE"] = "1" if request.param == "tile" else "0"
+    old = {k: os.environ.get(k) for k in ("B200ATTN_FP8_TILE", "B200ATTN_FP8_PAIR")}
+    tile, pair = FP8_KERNEL_ENV[request.param]
+    os.environ["B200ATTN_FP8_TILE"] = tile
+    os.environ["B200ATTN_FP8_PAIR"] = pair
     yield request.param
-    if old is None:
-        os.environ.pop("B200ATTN_FP8_TILE", None)
-    else:
-        os.environ["B200ATTN_FP8_TILE"] = old
+    for k, v in old.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
 
 
 # BF16 forms one exponential in four by a polynomial on the FMA pipe (default)
@@ -276,12 +281,13 @@ def test_fp8_many_units_per_cta(causal, fp8_p, fp8_kernel):
     assert err <= FP8_TOL, err
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "bf16-mixed", "fp8-lean", "fp8-mufu", "fp8-lean-tile"])
+@pytest.mark.parametrize("dtype", ["bf16", "bf16-mixed", "fp8-lean", "fp8-mufu", "fp8-lean-pair", "fp8-lean-tile"])
 def test_bitwise_deterministic_over_1000_launches(dtype, monkeypatch):
     monkeypatch.setenv("B200ATTN_BF16_P", "mixed" if dtype == "bf16-mixed" else "mufu")
     if dtype.startswith("fp8"):
         monkeypatch.setenv("B200ATTN_FP8_P", dtype.split("-")[1])
         monkeypatch.setenv("B200ATTN_FP8_TILE", "1" if dtype.endswith("-tile") else "0")
+        monkeypatch.setenv("B200ATTN_FP8_PAIR", "1" if dtype.endswith("-pair") else "0")
     q, k, v = workloads.draw(workloads.gaussian(1, 8, 2, 2048, 128, 128, seed=8))
     if dtype.startswith("bf16"):
         args = (q.cuda(), k.cuda(), v.cuda())
@@ -357,11 +363,11 @@ def test_full_size_fp8_sampled(name, hadamard, monkeypatch):
         assert_within(e, FP8_TOL)
 
 
-@pytest.mark.parametrize("fp8_kernel", ["tile"], indirect=True)
+@pytest.mark.parametrize("fp8_kernel", ["pair", "tile"], indirect=True)
 @pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
-def test_full_size_fp8_tile_kernel_sampled(fp8_p, fp8_kernel):
-    """The one-tile FP8 kernel on the full 7B-style layer (N = 16384), where its
-    K/V rings wrap many times per unit."""
+def test_full_size_fp8_other_kernels_sampled(fp8_p, fp8_kernel):
+    """The FP8 kernels other than the default on the full 7B-style layer
+    (N = 16384), where their K/V rings wrap many times per unit."""
     w = workloads.gqa7b()
     q, k, v = workloads.draw(w)
     heads, rows = sample_of(w)
@@ -369,7 +375,7 @@ def test_full_size_fp8_tile_kernel_sampled(fp8_p, fp8_kernel):
     ref8, _ = oracle_on_sample(*deq, heads, rows)
     o, _ = run_fp8(codes)
     e = error_report(gather_sample(o, heads, rows), ref8)
-    print(f"gqa7b fp8[{fp8_p}, one-tile kernel] {fmt_errors(e)}")
+    print(f"gqa7b fp8[{fp8_p}, {fp8_kernel} kernel] {fmt_errors(e)}")
     assert_within(e, FP8_TOL)
 
 
