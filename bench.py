@@ -56,6 +56,10 @@ def parse_args():
     ap.add_argument("--hadamard", action="store_true", help="rotate Q and K before FP8 quantisation")
     ap.add_argument("--energy-s", type=float, default=2.0,
                     help="seconds of back-to-back steps for the TFLOP/J figure (0: skip)")
+    ap.add_argument("--fp8-q", choices=["fused", "separate", "qblock"], default="qblock",
+                    help="FP8 step: Q quantised inside the attention kernel (fused, per 128-token tile), by the "
+                         "quantizer per head (separate), or by the quantizer per 128-token block in one pass "
+                         "(qblock); K and V per head by the quantizer")
     ap.add_argument("--fp8-p", choices=["lean", "mufu"], default=None,
                     help="how the FP8 kernel forms probabilities (default: the library default, Lean P)")
     ap.add_argument("--settle-s", type=float, default=1.0,
@@ -329,12 +333,20 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+def fp8_step_desc(args) -> str:
+    had = args.hadamard
+    if args.fp8_q == "fused":
+        return ("e4m3 quantizer on K,V (per-head scales" + (", Hadamard on K" if had else "")
+                + ") + FP8 attention quantising Q in the kernel (per-128-token scales" + (", Hadamard" if had else "")
+                + ")")
+    q = "per-128-token-block scales for Q, per-head for K,V" if args.fp8_q == "qblock" else "per-head scales"
+    return "e4m3 quantizer on Q,K,V (" + q + (", Hadamard on Q,K" if had else "") + ") + FP8 attention"
+
+
 def run_config(args, w: workloads.Workload, world: int) -> dict:
     """The `config` object of the JSON line; both arms print the same one."""
     return {"workload": workload_desc(w),
-            "step": ("e4m3 quantizer on Q,K,V (per-head scales"
-                     + (", Hadamard on Q,K" if args.hadamard else "") + ") + FP8 attention")
-            if args.dtype == "fp8" else "BF16 attention",
+            "step": fp8_step_desc(args) if args.dtype == "fp8" else "BF16 attention",
             "flops_per_step": w.flops, "flop_convention": "B*Hq*N^2*(d_qk+d_v)",
             "l2": "256 MiB buffer written between timed steps (untimed); inputs exceed L2",
             "settle": f"{args.settle_s} s of untimed back-to-back steps before timing",
@@ -349,8 +361,11 @@ def run_config(args, w: workloads.Workload, world: int) -> dict:
 class Path:
     """Preallocated buffers and the step of the hot path for one dtype."""
 
-    def __init__(self, b2, q, k, v, dtype: str, hadamard: bool):
+    def __init__(self, b2, q, k, v, dtype: str, hadamard: bool, fp8_q: str = "fused"):
         self.b2, self.q, self.k, self.v, self.dtype, self.hadamard = b2, q, k, v, dtype, hadamard
+        self.fp8_q = fp8_q
+        self.fused_q = fp8_q == "fused"
+        self.gran = "q_block" if fp8_q == "qblock" else "head"
         B, N, Hq, dqk = q.shape
         Hkv, dv = k.shape[2], v.shape[3]
         dev = q.device
@@ -359,23 +374,32 @@ class Path:
             self.q8 = torch.empty(q.shape, dtype=torch.float8_e4m3fn, device=dev)
             self.k8 = torch.empty(k.shape, dtype=torch.float8_e4m3fn, device=dev)
             self.v8 = torch.empty(v.shape, dtype=torch.float8_e4m3fn, device=dev)
-            self.sq = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+            self.sq = torch.empty((B, Hq) if fp8_q != "qblock" else (B, Hq, -(-N // 128)), dtype=torch.float32,
+                                  device=dev)
             self.sk = torch.empty((B, Hkv), dtype=torch.float32, device=dev)
             self.sv = torch.empty((B, Hkv), dtype=torch.float32, device=dev)
-            ws = max(b2.quantize_qkv_workspace_bytes(B, N, Hq, Hkv), 4)
+            ws = max(b2.quantize_qkv_workspace_bytes(B, N, Hq, Hkv, self.gran), 4)
             self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
-        # FP8: absmax and encode passes over Q, K and V (one launch each), attention
+        # FP8: absmax and encode passes over K and V (with Q too when not fused; one
+        # launch each), attention
         self.launches_per_step = 3 if dtype == "fp8" else 1
 
     def step(self, ev_a0=None, ev_a1=None):
         b2 = self.b2
-        if self.dtype == "fp8":
-            b2.quantize_qkv_fp8(self.q, self.k, self.v, hadamard=self.hadamard, workspace=self.ws,
-                                out=(self.q8, self.sq, self.k8, self.sk, self.v8, self.sv))
+        if self.dtype == "fp8" and self.fused_q:
+            b2.quantize_kv_fp8(self.k, self.v, hadamard=self.hadamard, workspace=self.ws,
+                               out=(self.k8, self.sk, self.v8, self.sv))
+            if ev_a0 is not None:
+                ev_a0.record()
+            b2.attn_fwd_fused_q(self.q, self.k8, self.v8, k_scale=self.sk, v_scale=self.sv, hadamard=self.hadamard,
+                                out=self.o)
+        elif self.dtype == "fp8":
+            b2.quantize_qkv_fp8(self.q, self.k, self.v, granularity=self.gran, hadamard=self.hadamard,
+                                workspace=self.ws, out=(self.q8, self.sq, self.k8, self.sk, self.v8, self.sv))
             if ev_a0 is not None:
                 ev_a0.record()
             b2.attn_fwd(self.q8, self.k8, self.v8, q_scale=self.sq, k_scale=self.sk, v_scale=self.sv,
-                        out=self.o)
+                        scale_granularity=self.gran, out=self.o)
         else:
             if ev_a0 is not None:
                 ev_a0.record()
@@ -443,13 +467,18 @@ def measure_energy(clk, path, flops_per_step: float, seconds: float):
             "source": "NVML total energy consumption of this GPU over steps run back to back (no L2 flush)"}
 
 
-def quantizer_summary(quant_ms: float, w: workloads.Workload, hbm_peak: float) -> dict:
+# Quantizer bytes per element of Q: per head, two passes (2 + 2 read, 1 written);
+# per 128-token block, one pass (2 read, 1 written); none when the attention
+# kernel quantises Q itself.
+QUANT_Q_BYTES = {"separate": 5.0, "qblock": 3.0, "fused": 0.0}
+
+
+def quantizer_summary(quant_ms: float, w: workloads.Workload, hbm_peak: float, q_bytes: float = 5.0) -> dict:
     """The FP8 step's quantizer against the HBM roofline. quant_ms is the part of the step
     outside the attention kernel's events: the absmax and encode launches plus launch gaps.
-    Algorithmic bytes with per-head scales: a 2-byte read in each pass and a 1-byte write,
-    5 bytes per element of Q, K and V."""
-    elems = w.B * w.N * (w.Hq * w.d_qk + w.Hkv * (w.d_qk + w.d_v))
-    nbytes = 5.0 * elems
+    Algorithmic bytes: K and V per head, a 2-byte read in each of two passes and a 1-byte
+    write (5 bytes per element), plus q_bytes per element of Q."""
+    nbytes = w.B * w.N * (q_bytes * w.Hq * w.d_qk + 5.0 * w.Hkv * (w.d_qk + w.d_v))
     if not quant_ms > 0.0:
         return None
     gbs = nbytes / (quant_ms * 1e-3) / 1e9
@@ -467,8 +496,11 @@ def max_over_ranks(x: float, dist_on: bool, device: str = "cuda") -> float:
     return float(t.item())
 
 
-def kernel_name(dtype: str, w: workloads.Workload) -> str:
+def kernel_name(dtype: str, w: workloads.Workload, fused_q: bool = False) -> str:
     """The attention kernel (and probability mode) the library runs for this call."""
+    if dtype == "fp8" and fused_q:
+        fp8_p = "mufu" if os.environ.get("B200ATTN_FP8_P") == "mufu" else "lean"
+        return f"attn_fwd_kernel<{w.d_qk},{w.d_v},fp8,{fp8_p},fused-q>"
     if dtype == "fp8":
         fp8_p = "mufu" if os.environ.get("B200ATTN_FP8_P") == "mufu" else "lean"
         if os.environ.get("B200ATTN_FP8_TILE") == "1":
@@ -497,7 +529,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     fp8_peak, fp8_peak_src = load_fp8_peak(bf16_peak, peak_src)
 
     def measure(dtype, wl, tensors, clk=None):
-        path = Path(b2, *tensors, dtype, args.hadamard)
+        path = Path(b2, *tensors, dtype, args.hadamard, args.fp8_q)
         step_ms, attn_ms = time_path(path, args.steps, args.warmup, args.settle_s, flush, dist_on, clk)
         if b2.check() != 0:
             raise RuntimeError("a kernel reported a timeout")
@@ -506,7 +538,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         value = world * wl.flops / (ms * 1e-3) / 1e12
         achieved = wl.flops / (ams * 1e-3) / 1e12
         peak = fp8_peak if dtype == "fp8" else bf16_peak
-        kernel_key = kernel_name(dtype, wl)
+        kernel_key = kernel_name(dtype, wl, args.fp8_q == "fused")
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic_for(kernel_key, wl.name),
                 "kernel": kernel_key, "kernel_ms": ams,
@@ -515,7 +547,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         quant = None
         if dtype == "fp8":
             qms = max_over_ranks(statistics.mean([s - a for s, a in zip(step_ms, attn_ms)]), dist_on)
-            quant = quantizer_summary(qms, wl, hbm_peak)
+            quant = quantizer_summary(qms, wl, hbm_peak, q_bytes=QUANT_Q_BYTES[args.fp8_q])
         return {"value": value, "ms_per_step": ms, "roofline": roof, "quantizer": quant,
                 "launches": path.launches_per_step * args.steps,
                 "step_ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))]}
@@ -523,7 +555,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     with ClockSampler(local_rank) as clk:
         main = measure(args.dtype, w, (q, k, v), clk)
     clocks = clk.summary()
-    energy = measure_energy(clk, Path(b2, q, k, v, args.dtype, args.hadamard), w.flops, args.energy_s)
+    energy = measure_energy(clk, Path(b2, q, k, v, args.dtype, args.hadamard, args.fp8_q), w.flops, args.energy_s)
     other = None
     if not args.no_other_dtype:
         other_dtype = "bf16" if args.dtype == "fp8" else "fp8"
@@ -585,7 +617,7 @@ def measure_e2e(b2, args, w, q_cpu, k_cpu, v_cpu, world, dist_on):
     q = torch.empty_like(q_cpu, device="cuda")
     k = torch.empty_like(k_cpu, device="cuda")
     v = torch.empty_like(v_cpu, device="cuda")
-    path = Path(b2, q, k, v, args.dtype, args.hadamard)
+    path = Path(b2, q, k, v, args.dtype, args.hadamard, args.fp8_q)
 
     def step():
         q.copy_(hq, non_blocking=True)

@@ -8,11 +8,14 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     attn_func,
     attn_fwd,
+    attn_fwd_fused_q,
     attn_varlen_func,
     attn_varlen_fwd,
     check,
     load_library,
     quantize_fp8,
+    quantize_kv_fp8,
+    quantize_kv_workspace_bytes,
     quantize_qkv_fp8,
     quantize_qkv_workspace_bytes,
     quantize_workspace_bytes,

@@ -19,7 +19,9 @@ BF16 = 0
 FP8_E4M3 = 1
 SCALE_PER_HEAD = 0
 SCALE_PER_BLOCK = 1
-_GRAN = {"head": SCALE_PER_HEAD, "block": SCALE_PER_BLOCK}
+SCALE_Q_BLOCK = 2
+# "q_block": Q's scales per 128-token block, K's and V's per head
+_GRAN = {"head": SCALE_PER_HEAD, "block": SCALE_PER_BLOCK, "q_block": SCALE_Q_BLOCK}
 BLOCK = 128
 
 _lib = None
@@ -68,6 +70,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.b200attn_selftest_wait_timeout.argtypes = [i, vp]
     lib.b200attn_trace_read.restype = i
     lib.b200attn_trace_read.argtypes = [vp, i, i, i]
+    lib.b200attn_fwd_fp8_fused_q.restype = i
+    lib.b200attn_fwd_fp8_fused_q.argtypes = [vp, vp, vp, vp] + [i] * 7 + [vp, vp, i, f, vp, vp, vp, vp]
+    lib.b200attn_quantize_kv_workspace_bytes.restype = sz
+    lib.b200attn_quantize_kv_workspace_bytes.argtypes = [i, i, i, i]
+    lib.b200attn_quantize_kv_fp8.restype = i
+    lib.b200attn_quantize_kv_fp8.argtypes = [vp] * 6 + [i] * 7 + [vp, sz, vp]
     _lib = lib
     return lib
 
@@ -111,12 +119,14 @@ def _check_buffer(name, t, shape, dtypes, device):
 
 def _gran(granularity: str) -> int:
     if granularity not in _GRAN:
-        raise ValueError("granularity must be 'head' or 'block'")
+        raise ValueError("granularity must be 'head', 'block' or 'q_block'")
     return _GRAN[granularity]
 
 
-def _scale_shape(B: int, H: int, N: int, granularity: str):
-    return (B, H) if granularity == "head" else (B, H, math.ceil(N / BLOCK))
+def _scale_shape(B: int, H: int, N: int, granularity: str, tensor: str = "q"):
+    """Shape of tensor `tensor`'s ("q", "k" or "v") scales at this granularity."""
+    per_block = granularity == "block" or (granularity == "q_block" and tensor == "q")
+    return (B, H, math.ceil(N / BLOCK)) if per_block else (B, H)
 
 
 def _check_scale(name, s, B, H, N, granularity, device):
@@ -124,7 +134,7 @@ def _check_scale(name, s, B, H, N, granularity, device):
     tensor with that many elements is accepted too."""
     if s is None:
         raise ValueError(f"{name} is required for e4m3 inputs")
-    shape = _scale_shape(B, H, N, granularity)
+    shape = _scale_shape(B, H, N, granularity, name[0])
     if isinstance(s, torch.Tensor) and s.dim() == 1 and s.numel() == math.prod(shape):
         shape = (s.numel(),)
     _check_buffer(name, s, shape, (torch.float32,), device)
@@ -258,6 +268,8 @@ def quantize_fp8(x, *, granularity: str = "head", hadamard: bool = False, out=No
     if x.dtype != torch.bfloat16 or x.dim() != 4:
         raise ValueError("x must be bf16 [B, N, H, d]")
     B, N, H, d = x.shape
+    if granularity not in ("head", "block"):
+        raise ValueError("granularity of one tensor must be 'head' or 'block'")
     gran = _gran(granularity)
     if out is None:
         out = torch.empty((B, N, H, d), dtype=torch.float8_e4m3fn, device=x.device)
@@ -304,13 +316,15 @@ def quantize_qkv_fp8(q, k, v, *, granularity: str = "head", hadamard: bool = Fal
         out = []
         for t, H in ((q, Hq), (k, Hkv), (v, Hkv)):
             out.append(torch.empty(t.shape, dtype=torch.float8_e4m3fn, device=dev))
-            out.append(torch.empty(_scale_shape(B, H, N, granularity), dtype=torch.float32, device=dev))
+            out.append(torch.empty(_scale_shape(B, H, N, granularity, "q" if t is q else "k"), dtype=torch.float32,
+                                   device=dev))
     else:
         if len(out) != 6:
             raise ValueError("out must hold six tensors: q8, q_scale, k8, k_scale, v8, v_scale")
         for i, (name, t, H) in enumerate((("q", q, Hq), ("k", k, Hkv), ("v", v, Hkv))):
             _check_buffer(f"{name}8", out[2 * i], tuple(t.shape), _E4M3_DTYPES, dev)
-            _check_buffer(f"{name}_scale", out[2 * i + 1], _scale_shape(B, H, N, granularity), (torch.float32,), dev)
+            _check_buffer(f"{name}_scale", out[2 * i + 1], _scale_shape(B, H, N, granularity, name), (torch.float32,),
+                          dev)
     q8, sq, k8, sk, v8, sv = out
     need = quantize_qkv_workspace_bytes(B, N, Hq, Hkv, granularity)
     if workspace is None and need > 0:
@@ -324,17 +338,115 @@ def quantize_qkv_fp8(q, k, v, *, granularity: str = "head", hadamard: bool = Fal
     return q8, sq, k8, sk, v8, sv
 
 
+def quantize_kv_workspace_bytes(B, N, Hkv, granularity="head") -> int:
+    return int(load_library().b200attn_quantize_kv_workspace_bytes(B, N, Hkv, _gran(granularity)))
+
+
+def quantize_kv_fp8(k, v, *, granularity: str = "head", hadamard: bool = False, out=None, workspace=None,
+                    stream=None):
+    """bf16 K, V -> (k8, sk, v8, sv) through b200attn_quantize_kv_fp8 (the rotation,
+    with ``hadamard``, on K only). ``out`` may pass the four output tensors."""
+    lib = load_library()
+    for name, t in (("k", k), ("v", v)):
+        _check_cuda_contig(name, t)
+        if t.dtype != torch.bfloat16 or t.dim() != 4:
+            raise ValueError(f"{name} must be bf16 [B, N, H, d]")
+    B, N, Hkv, d_qk = k.shape
+    d_v = v.shape[3]
+    if v.shape != (B, N, Hkv, d_v):
+        raise ValueError("shape mismatch between k and v")
+    if granularity not in ("head", "block"):
+        raise ValueError("granularity of K and V must be 'head' or 'block'")
+    gran = _gran(granularity)
+    dev = k.device
+    if v.device != dev:
+        raise ValueError("k and v must be on one device")
+    if out is None:
+        out = []
+        for t in (k, v):
+            out.append(torch.empty(t.shape, dtype=torch.float8_e4m3fn, device=dev))
+            out.append(torch.empty(_scale_shape(B, Hkv, N, granularity), dtype=torch.float32, device=dev))
+    else:
+        if len(out) != 4:
+            raise ValueError("out must hold four tensors: k8, k_scale, v8, v_scale")
+        for i, (name, t) in enumerate((("k", k), ("v", v))):
+            _check_buffer(f"{name}8", out[2 * i], tuple(t.shape), _E4M3_DTYPES, dev)
+            _check_buffer(f"{name}_scale", out[2 * i + 1], _scale_shape(B, Hkv, N, granularity), (torch.float32,),
+                          dev)
+    k8, sk, v8, sv = out
+    need = quantize_kv_workspace_bytes(B, N, Hkv, granularity)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.b200attn_quantize_kv_fp8(_ptr(k), _ptr(v), _ptr(k8), _ptr(v8), _ptr(sk), _ptr(sv), B, N, Hkv, d_qk,
+                                      d_v, gran, 1 if hadamard else 0, _ptr(workspace), wbytes,
+                                      _stream_handle(stream))
+    if rc != 0:
+        raise B200AttnError(rc, "b200attn_quantize_kv_fp8")
+    return k8, sk, v8, sv
+
+
+def attn_fwd_fused_q(q, k8, v8, *, k_scale, v_scale, causal: bool = True, softmax_scale: float | None = None,
+                     hadamard: bool = False, out=None, return_lse: bool = False, q_out=None, q_scale_out=None,
+                     stream=None):
+    """FP8 attention with Q in bf16, quantised inside the kernel (one scale per
+    128-token block of each head), via b200attn_fwd_fp8_fused_q. k8, v8 are e4m3
+    with per-head scales [B, Hkv]. ``q_out`` / ``q_scale_out`` (optional) receive
+    the codes [B,N,Hq,d_qk] and scales [B,Hq,ceil(N/128)] the kernel used."""
+    lib = load_library()
+    _check_cuda_contig("q", q)
+    if q.dtype != torch.bfloat16 or q.dim() != 4:
+        raise ValueError("q must be bf16 [B, N, H, d]")
+    for name, t in (("k8", k8), ("v8", v8)):
+        _check_cuda_contig(name, t)
+        if not _is_fp8(t) or t.dim() != 4:
+            raise ValueError(f"{name} must be e4m3 [B, N, H, d]")
+    B, N, Hq, d_qk = q.shape
+    Hkv, d_v = k8.shape[2], v8.shape[3]
+    if k8.shape != (B, N, Hkv, d_qk) or v8.shape != (B, N, Hkv, d_v):
+        raise ValueError("shape mismatch between q, k and v")
+    dev = q.device
+    if k8.device != dev or v8.device != dev:
+        raise ValueError("q, k and v must be on one device")
+    _check_scale("k_scale", k_scale, B, Hkv, N, "head", dev)
+    _check_scale("v_scale", v_scale, B, Hkv, N, "head", dev)
+    if out is None:
+        out = torch.empty((B, N, Hq, d_v), dtype=torch.bfloat16, device=dev)
+    else:
+        _check_buffer("out", out, (B, N, Hq, d_v), (torch.bfloat16,), dev)
+    if q_out is not None:
+        _check_buffer("q_out", q_out, (B, N, Hq, d_qk), _E4M3_DTYPES, dev)
+    if q_scale_out is not None:
+        _check_buffer("q_scale_out", q_scale_out, _scale_shape(B, Hq, N, "block"), (torch.float32,), dev)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev) if return_lse else None
+    rc = lib.b200attn_fwd_fp8_fused_q(
+        _ptr(q), _ptr(k8), _ptr(v8), _ptr(out), B, Hq, Hkv, N, d_qk, d_v, 1 if causal else 0,
+        _ptr(k_scale), _ptr(v_scale), 1 if hadamard else 0, float(softmax_scale) if softmax_scale else 0.0,
+        _ptr(lse), _ptr(q_out), _ptr(q_scale_out), _stream_handle(stream))
+    if rc != 0:
+        raise B200AttnError(rc, "b200attn_fwd_fp8_fused_q")
+    return (out, lse) if return_lse else out
+
+
 def attn_func(q, k, v, softmax_scale: float | None = None, causal: bool = True, *, fp8: bool = False,
-              hadamard: bool = False, granularity: str = "head", return_lse: bool = False, stream=None):
+              hadamard: bool = False, granularity: str = "q_block", fused_q: bool = False, return_lse: bool = False,
+              stream=None):
     """flash_attn_func-style call on bf16 [B,N,H,d] tensors.
 
     With ``fp8=True`` Q, K and V are first quantised to e4m3 (Q and K
-    optionally Hadamard-rotated, which leaves Q K^T unchanged), then the FP8
-    kernel runs.
+    optionally Hadamard-rotated, which leaves Q K^T unchanged) at
+    ``granularity``: by default Q per 128-token block (one pass) and K, V per
+    head; "head" or "block" for all three. Then the FP8 kernel runs. With
+    ``fused_q=True`` only K and V are quantised first (per head) and the
+    attention kernel quantises Q itself, per 128-token block.
     """
     if not fp8:
         return attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale, return_lse=return_lse,
                         stream=stream)
+    if fused_q:
+        k8, sk, v8, sv = quantize_kv_fp8(k, v, hadamard=hadamard, stream=stream)
+        return attn_fwd_fused_q(q, k8, v8, k_scale=sk, v_scale=sv, causal=causal, softmax_scale=softmax_scale,
+                                hadamard=hadamard, return_lse=return_lse, stream=stream)
     q8, sq, k8, sk, v8, sv = quantize_qkv_fp8(q, k, v, granularity=granularity, hadamard=hadamard, stream=stream)
     return attn_fwd(q8, k8, v8, causal=causal, softmax_scale=softmax_scale, q_scale=sq, k_scale=sk,
                     v_scale=sv, scale_granularity=granularity, return_lse=return_lse, stream=stream)

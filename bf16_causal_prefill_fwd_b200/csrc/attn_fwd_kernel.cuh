@@ -84,6 +84,7 @@
 #include <cuda_bf16.h>
 
 #include "attn_trace.cuh"
+#include "q_encode.cuh"
 #include "sm100_ptx.cuh"
 
 namespace b200 {
@@ -114,7 +115,8 @@ struct AttnParams {
   int n_pairs;   // ceil(n_kv / 2)
   int n_units;   // B * Hq * n_pairs
   int causal;
-  int per_block;  // FP8 scales per 128-token block (else per head)
+  int per_block;    // FP8 scales of Q, K and V per 128-token block (else per head)
+  int q_per_block;  // FP8, per_block == 0: Q's scales per 128-token block, K's and V's per head
   float scale_log2;
   const float* q_scale;
   const float* k_scale;
@@ -125,9 +127,17 @@ struct AttnParams {
   // along the token dimension (B = 1, N = total tokens) and units are read from
   // this table, already ordered longest first.
   const VarlenUnit* units;
+  // FP8 with Q quantised in the kernel (template flag QF): Q as bf16, one scale
+  // per (b, h, 128-token tile) computed there, optional Hadamard rotation of
+  // the rows; the codes and scales are also written out when the pointers are
+  // set (e4m3 [B, N, Hq, d_qk] and fp32 [B, Hq, n_kv]).
+  const __nv_bfloat16* q_bf16;
+  int q_hadamard;
+  uint8_t* q_codes_out;
+  float* q_scale_out;
 };
 
-template <int DQK, int DV, bool FP8, bool FMA_P = false, bool SHARED_S = true>
+template <int DQK, int DV, bool FP8, bool FMA_P = false, bool SHARED_S = true, bool QF = false>
 struct AttnCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int CHUNK_ELEMS = 128 / ESZ;  // elements in one 128-byte swizzled row
@@ -157,13 +167,18 @@ struct AttnCfg {
   static constexpr int ONES_BYTES = RS ? CHUNK_BYTES : 0;
   // Separate K and V rings, sized from what shared memory has left.
   static constexpr int SMEM_AVAIL = 227 * 1024 - 2048;  // minus barriers and alignment slack
-  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BYTES - ONES_BYTES;
+  // Q buffers per tile. With two (QF only) the next unit's Q tile could be
+  // written while the current one is in use; measured, that was slower than
+  // writing it between units (the encode then sits in the middle of the
+  // softmax's pipeline and the K ring loses a stage), so one is used.
+  static constexpr int Q_BUFS = 1;
+  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BUFS * Q_BYTES - ONES_BYTES;
   static constexpr int RING_PAIRS = RING_AVAIL / (K_BYTES + V_BYTES);
   static constexpr int SV = RING_PAIRS >= 2 ? (RING_PAIRS > 4 ? 4 : RING_PAIRS) : 1;
   static constexpr int SK_FIT = (RING_AVAIL - SV * V_BYTES) / K_BYTES;
   static constexpr int SK = SK_FIT > 6 ? 6 : SK_FIT;
-  static constexpr int NUM_BARS = 2 + 2 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
-  static constexpr int SMEM_BYTES = 2 * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES +
+  static constexpr int NUM_BARS = 4 + 4 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
+  static constexpr int SMEM_BYTES = 2 * Q_BUFS * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES +
                                     1024 /*bars*/ + 1024 /*align*/;
   static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
   static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
@@ -172,7 +187,7 @@ struct AttnCfg {
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
   static_assert(SK >= 2 && SV >= 1, "K/V rings");
   static_assert(!SS || TM_P + 2 * PB * P_COLS <= 512, "TMEM budget");
-  static_assert(8 * NUM_BARS + 8 <= 1024, "barrier area");
+  static_assert(8 * NUM_BARS + 8 <= 512, "barrier area (the Q-encode reduction sits at +512)");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -267,11 +282,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort_flag);
 }
 
-template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S>
+template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S, bool QF = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S>;
+  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S, QF>;
+  static_assert(!QF || (FP8 && SHARED_S), "Q is quantised in the kernel only on the FP8 shared-S path");
   extern __shared__ uint8_t smem_raw[];
 
   // 1024-byte aligned base (128-byte swizzle atoms repeat every 1024 bytes).
@@ -280,7 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* base = smem_raw + (base_u32 - raw_u32);
 
   const uint32_t sQ = base_u32;                              // 2 query tiles
-  const uint32_t sK = sQ + 2 * C::Q_BYTES;                   // K ring
+  const uint32_t sK = sQ + 2 * C::Q_BUFS * C::Q_BYTES;       // K ring
   const uint32_t sV = sK + C::SK * C::K_BYTES;               // V ring
   const uint32_t sOnes = sV + C::SV * C::V_BYTES;          // RS: e4m3 ones, B columns d_v..d_v+15
   const uint32_t sBar = sOnes + C::ONES_BYTES;
@@ -289,9 +305,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NUM_BARS + 4);
 
   // barrier addresses
-  const uint32_t bQFull = sBar;                          // [2]  TMA -> QK issuer
-  const uint32_t bQEmpty = bQFull + 16;                  // [2]  QK issuer -> TMA
-  const uint32_t bKFull = bQEmpty + 16;                  // [SK] TMA -> QK issuer
+  // Q tile t, buffer qb (QF: unit k uses qb = k % 2; otherwise always 0) at
+  // sQ + (t * Q_BUFS + qb) * Q_BYTES, its barriers at index 2 t + qb.
+  const uint32_t bQFull = sBar;                          // [2][2] TMA (or the tile's softmax, QF) -> QK issuer
+  const uint32_t bQEmpty = bQFull + 32;                  // [2][2] QK issuer -> TMA (or softmax)
+  const uint32_t bKFull = bQEmpty + 32;                  // [SK] TMA -> QK issuer
   const uint32_t bKEmpty = bKFull + 8 * C::SK;           // [SK] QK issuer -> TMA
   const uint32_t bVFull = bKEmpty + 8 * C::SK;           // [SV] TMA -> PV issuer
   const uint32_t bVEmpty = bVFull + 8 * C::SV;           // [SV] PV issuer -> TMA
@@ -315,8 +333,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       for (int t = 0; t < 2; ++t) {
-        mbar_init(bQFull + 8 * t, 1);
-        mbar_init(bQEmpty + 8 * t, 1);
+        for (int qb = 0; qb < 2; ++qb) {
+          mbar_init(bQFull + 8 * (2 * t + qb), QF ? 128 : 1);  // QF: the tile's softmax threads write Q
+          mbar_init(bQEmpty + 8 * (2 * t + qb), 1);
+        }
         mbar_init(bSFull + 8 * t, 1);
         if (t == 0) mbar_init(bSFree, 128);
         for (int b = 0; b < C::PBX; ++b) {
@@ -383,14 +403,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int u = unit_for(k, blockIdx.x, gridDim.x);
         if (u >= p.n_units) break;
         const Unit x = decode_unit(u, p);
-        if (is_k) {
+        if (is_k && !QF) {
           for (int t = 0; t < 2 && ok; ++t) {
             if (!first) {
-              ok = mbar_wait(bQEmpty + 8 * t, qe_par[t], abort_flag);
+              ok = mbar_wait(bQEmpty + 16 * t, qe_par[t], abort_flag);
               qe_par[t] ^= 1;
               if (!ok) break;
             }
-            const uint32_t bar = bQFull + 8 * t;
+            const uint32_t bar = bQFull + 16 * t;
             mbar_arrive_expect_tx(bar, C::Q_BYTES);
 #pragma unroll
             for (int c = 0; c < C::QK_CHUNKS; ++c)
@@ -427,8 +447,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint32_t oe_par[2] = {0, 0};
       bool first = true, ok = true;
       // QK^T for tile t into S_t from K slot s.
-      auto issue_qk = [&](int t, uint32_t s) {
-        const uint32_t a_lo = q_lo0 + t * (C::Q_BYTES >> 4);
+      auto issue_qk = [&](int t, uint32_t s, uint32_t qb) {
+        const uint32_t a_lo = q_lo0 + (t * C::Q_BUFS + qb) * (C::Q_BYTES >> 4);
         const uint32_t b_lo = k_lo0 + s * (C::K_BYTES >> 4);
 #pragma unroll
         for (int kk = 0; kk < DQK / C::MMA_K; ++kk) {
@@ -468,7 +488,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // previous S out. Warp 2: O_t += P_t(j) V_j once the softmax has written
           // P_t(j) (and rescaled O_t).
           if (warp == 1) {
-            ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
+            const uint32_t qb = C::Q_BUFS == 2 ? (k & 1) : 0;
+            const uint32_t qpar = C::Q_BUFS == 2 ? ((k >> 1) & 1) : q_par;
+            ok = mbar_wait(bQFull + 8 * qb, qpar, abort_flag) && mbar_wait(bQFull + 8 * (2 + qb), qpar, abort_flag);
             if (!ok) break;
             q_par ^= 1;
             for (int j = 0; j < x.n1 && ok; ++j) {
@@ -481,9 +503,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 trace(kEvQkIssue, nq);
                 ++nq;
                 tc_fence_after();
-                issue_qk(t, s);
+                issue_qk(t, s, qb);
                 tc_commit(bSFull + 8 * t);
-                if (j == n_t - 1) tc_commit(bQEmpty + 8 * t);
+                if (j == n_t - 1) tc_commit(bQEmpty + 8 * (2 * t + qb));
               }
               if (!ok) break;
               tc_commit(bKEmpty + 8 * s);
@@ -519,16 +541,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // order, so PV_t(j-1) has read P (in S_t's columns) before S_t(j)
           // overwrites them, and each tile's PV and next QK^T run back to back.
           if (warp != 1) break;
-          ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 8, q_par, abort_flag);
+          ok = mbar_wait(bQFull, q_par, abort_flag) && mbar_wait(bQFull + 16, q_par, abort_flag);
           if (!ok) break;
           q_par ^= 1;
           uint32_t ks;
           if (!(ok = take(bKFull, C::SK, kit, ks))) break;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
-            issue_qk(t, ks);
+            issue_qk(t, ks, 0);
             tc_commit(bSFull + 8 * t);
-            if ((t ? x.n1 : x.n0) == 1) tc_commit(bQEmpty + 8 * t);
+            if ((t ? x.n1 : x.n0) == 1) tc_commit(bQEmpty + 16 * t);
           }
           tc_commit(bKEmpty + 8 * ks);
           for (int i = 1; i <= x.n1 && ok; ++i) {
@@ -553,9 +575,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tc_fence_after();
               }
               if (i < n_t) {
-                issue_qk(t, ks);
+                issue_qk(t, ks, 0);
                 tc_commit(bSFull + 8 * t);
-                if (i == n_t - 1) tc_commit(bQEmpty + 8 * t);
+                if (i == n_t - 1) tc_commit(bQEmpty + 16 * t);
               }
             }
             if (!ok) break;
@@ -594,6 +616,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const bool tracer = (warp & 3) == 0 && lane == 0;  // one thread per softmax warpgroup logs events
     bool ok = true;
 
+    // QF: this warpgroup quantises its own Q tile of every unit (q_encode.cuh),
+    // one thread per row: the rows are prefetched into L2 after the unit
+    // before's last probabilities, and encoded after its epilogue, once its
+    // last QK^T of the tile has read the Q buffer.
+    float sq_tile = 1.0f;  // scale of this warpgroup's Q tile in the current unit
+    float sq_next = 1.0f;  // ... in the next unit
+    float* q_red = reinterpret_cast<float*>(bar_ptr + 512) + 8 * t;  // [unit parity][4 warps] tile maxima
+    auto q_row_ptr = [&](const Unit& y) -> const __nv_bfloat16* {
+      const int row = (2 * y.pair + t) * kBM + r;
+      return row < y.len ? p.q_bf16 + ((static_cast<size_t>(y.b) * p.N + y.row0 + row) * p.Hq + y.hq) * DQK
+                         : nullptr;
+    };
+    auto q_finish = [&](const Unit& y, int ku) {  // encodes unit ku's Q row, arrives on QFull[t]
+      const uint32_t qbuf = C::Q_BUFS == 2 ? (ku & 1) : 0;
+      QRowRaw<DQK> q_raw;
+      q_row_load<DQK>(q_row_ptr(y), q_raw);
+      float* red = q_red + 4 * (ku & 1);
+      auto tile_amax = [&](float m) {  // max over the warpgroup's 128 rows
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[warp & 3] = m;
+        named_bar_sync(1 + t, 128);
+        return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      };
+      const int qt = 2 * y.pair + t, row = qt * kBM + r;
+      uint8_t* gout = (p.q_codes_out != nullptr && row < y.len)
+                          ? p.q_codes_out + ((static_cast<size_t>(y.b) * p.N + y.row0 + row) * p.Hq + y.hq) * DQK
+                          : nullptr;
+      float inv, scale;
+      if (p.q_hadamard) {
+        float v[DQK];
+        q_scale_pair(tile_amax(q_row_values<DQK, true>(q_raw, v)), inv, scale);
+        q_row_store<DQK>(v, inv, sQ + (t * C::Q_BUFS + qbuf) * C::Q_BYTES, r, C::CHUNK_BYTES, gout);
+      } else {
+        q_scale_pair(tile_amax(q_row_absmax_raw<DQK>(q_raw)), inv, scale);
+        q_row_store_raw<DQK>(q_raw, inv, sQ + (t * C::Q_BUFS + qbuf) * C::Q_BYTES, r, C::CHUNK_BYTES, gout);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bQFull + 8 * (2 * t + qbuf));
+      if (p.q_scale_out != nullptr && r == 0 && qt * kBM < y.len)
+        p.q_scale_out[(static_cast<size_t>(y.b) * p.Hq + y.hq) * p.n_kv + qt] = scale;
+      sq_next = scale;
+    };
+    if constexpr (QF) {
+      const int u0 = unit_for(0, blockIdx.x, gridDim.x);
+      if (u0 < p.n_units) {
+        q_finish(decode_unit(u0, p), 0);
+      }
+    }
+
     for (int k = 0; ok; ++k) {
       const int u = unit_for(k, blockIdx.x, gridDim.x);
       if (u >= p.n_units) break;
@@ -601,6 +673,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int n_t = t ? x.n1 : x.n0;
       const int q_tile = 2 * x.pair + t;
       const int qrow = q_tile * kBM + r;
+      const int u_next = unit_for(k + 1, blockIdx.x, gridDim.x);  // QF
+      if constexpr (QF) sq_tile = sq_next;
 
       // FP8 scales. Per head: one multiplier on S and one on O. Per 128-token
       // block: S of block i takes sq[q tile] * sk[i]; V's block scale sv[i] is
@@ -617,7 +691,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ks_blk = p.k_scale + kv_row;
           vs_blk = p.v_scale + kv_row;
         } else {
-          c_log2 *= __ldg(p.q_scale + x.b * p.Hq + x.hq) * __ldg(p.k_scale + x.b * p.Hkv + x.hkv);
+          const float sq = QF ? sq_tile
+                              : __ldg(p.q_scale + (p.q_per_block
+                                                       ? static_cast<size_t>(x.b * p.Hq + x.hq) * p.n_kv + q_tile
+                                                       : static_cast<size_t>(x.b * p.Hq + x.hq)));
+          c_log2 *= sq * __ldg(p.k_scale + x.b * p.Hkv + x.hkv);
           v_mult = __ldg(p.v_scale + x.b * p.Hkv + x.hkv);
         }
       }
@@ -865,6 +943,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_before();
         mbar_arrive(bPFull + 8 * (t * C::PBX + g % C::PBX));
         if (tracer) trace(kEvSoftmaxPDone, g);
+        if constexpr (QF) {
+          // the next unit's Q rows travel to L2 while the epilogue waits for O
+          if (i == n_t - 1 && u_next < p.n_units) q_row_prefetch<DQK>(q_row_ptr(decode_unit(u_next, p)));
+        }
       }
       if (!ok) break;
 
@@ -905,6 +987,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(bOe);
       if (tracer) trace(kEvEpilogue, g);
+      if constexpr (QF) {
+        if (u_next < p.n_units) {
+          // one Q buffer: free once this unit's last QK^T of the tile has read it
+          ok = __all_sync(0xffffffffu, mbar_wait(bQEmpty + 16 * t, k & 1, abort_flag));
+          if (!ok) break;
+          q_finish(decode_unit(u_next, p), k + 1);
+        }
+      }
+
     }
   }
 

@@ -38,7 +38,7 @@
 // Tensor memory per SM (512 columns, the same addresses in both CTAs):
 //   [0,128) S buffer 0  [128,256) S buffer 1  (key block g uses g % 2)
 //   [256,416) O (160 columns as above)
-//   [416,448) P buffer 0  [448,480) P buffer 1  (e4m3 codes, 4 per column)
+//   [416,512) P buffers 0, 1, 2 (block g uses g % 3; e4m3 codes, 4 per column)
 //
 // Warp roles (384 threads per CTA):
 //   warp 0      TMA: this CTA's Q tile (double-buffered per unit) and K halves
@@ -72,10 +72,11 @@ struct PairCfg {
   static constexpr int MMA_K = 32;
   static constexpr int N_PV = 160;                      // 2 x (64 value columns + 16 ones)
   static constexpr int TM_O = 256, TM_P = 416, P_COLS = 32;
+  static constexpr int PB = 3;                          // P buffers: P(g) waits for PV(g-3) only
   static constexpr int O_HALF = 80;                     // D columns per CTA-half of B
   static constexpr int SMEM_AVAIL = 227 * 1024 - 2048;
   static constexpr int SK = 6, SV = 6;
-  static constexpr int NUM_BARS = 2 + 2 + 2 * SK + 2 * SV + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 2;
+  static constexpr int NUM_BARS = 2 + 2 + 2 * SK + 2 * SV + 2 + 2 + PB + PB + 2 + 2 + 1 + 2;
   static constexpr int XM_BYTES = 2 * kBM * 4;         // running max handed between the groups
   static constexpr int SMEM_BYTES =
       2 * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES + 1024 /*bars*/ + XM_BYTES + 1024 /*align*/;
@@ -84,20 +85,28 @@ struct PairCfg {
   static constexpr uint32_t IDESC_QK = idesc_dense(0u, 0u, 256, kBN, false);
   static constexpr uint32_t IDESC_PV = idesc_dense(0u, 0u, 256, N_PV, true);
   static_assert(DV == 128, "d_v = 128");
-  static_assert(TM_O + N_PV <= TM_P && TM_P + 2 * P_COLS <= 512, "TMEM budget");
+  static_assert(TM_O + N_PV <= TM_P && TM_P + PB * P_COLS <= 512, "TMEM budget");
   static_assert(8 * NUM_BARS + 8 <= 1024, "barrier area");
   static_assert(SMEM_BYTES <= SMEM_AVAIL + 2048, "shared memory budget");
 };
 
-// Bounded wait with cluster-scope acquire (the phase may be completed by the
-// other CTA of the pair). Same contract as mbar_wait.
+// Bounded wait on a barrier the other CTA of the pair may complete: the same
+// wait as mbar_wait (what it orders is tensor-memory access, fenced by tcgen05
+// fences on both sides).
 __device__ __forceinline__ bool pair_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort_flag);
+}
+
+// The same for the single-thread roles (issuers, producers), by polling with
+// a non-blocking test: in the per-block trace a suspended try_wait saw a phase
+// that arrivals from the other CTA completed only ~1700-2000 cycles late.
+__device__ __forceinline__ bool pair_wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 256; ++i)
-      if (mbar_try_wait_cluster(bar, parity)) return true;
+    for (int i = 0; i < 1024; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -147,9 +156,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   const uint32_t bVEmpty = bVFull + 8 * C::SV;        // [SV] both
   const uint32_t bSFull = bVEmpty + 8 * C::SV;        // [2]  both: S of block g in buffer g % 2
   const uint32_t bSFree = bSFull + 16;                // [2]  leader: 8 warps copied S out
-  const uint32_t bPFull = bSFree + 16;                // [2]  leader: 8 warps wrote P
-  const uint32_t bPDone = bPFull + 16;                // [2]  both: PV of the block done
-  const uint32_t bMReady = bPDone + 16;               // [2]  local: running max of block g published (128)
+  const uint32_t bPFull = bSFree + 16;                // [PB] leader: 8 warps wrote P into buffer g % PB
+  const uint32_t bPDone = bPFull + 8 * C::PB;         // [PB] both: PV of the block done
+  const uint32_t bMReady = bPDone + 8 * C::PB;        // [2]  local: running max of block g published (128)
   // O of unit k complete: one barrier per unit parity, since the group that
   // writes unit k's output may not have seen unit k-1's completion.
   const uint32_t bOFull = bMReady + 16;               // [2]  both
@@ -173,13 +182,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         mbar_init(bQEmpty + 8 * i, 1);
         mbar_init(bSFull + 8 * i, 1);
         mbar_init(bSFree + 8 * i, 8);
-        mbar_init(bPFull + 8 * i, 8);
-        mbar_init(bPDone + 8 * i, 1);
         mbar_init(bMReady + 8 * i, 128);
         mbar_init(bDrain + 8 * i, 1);
         mbar_init(bOFull + 8 * i, 1);
       }
       mbar_init(bOEmpty, 8);
+      for (int i = 0; i < C::PB; ++i) {
+        mbar_init(bPFull + 8 * i, 8);
+        mbar_init(bPDone + 8 * i, 1);
+      }
       for (int s = 0; s < C::SK; ++s) {
         mbar_init(bKFull + 8 * s, 1);
         mbar_init(bKEmpty + 8 * s, 1);
@@ -233,7 +244,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           const Unit x = decode_unit(u, p);
           if (is_k) {
             const uint32_t qb = k & 1;
-            if (k >= 2 && !(ok = pair_wait(bQEmpty + 8 * qb, ((k - 2) >> 1) & 1, abort_flag))) break;
+            if (k >= 2 && !(ok = pair_wait_spin(bQEmpty + 8 * qb, ((k - 2) >> 1) & 1, abort_flag))) break;
             const uint32_t bar = bQFull + 8 * qb;
             if (rank == 0) mbar_arrive_expect_tx(bar, 2 * C::Q_BYTES);
 #pragma unroll
@@ -244,7 +255,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           for (int j = 0; j < x.n1 && ok; ++j, ++it) {
             const uint32_t s = it % nslot;
             if (it >= static_cast<uint32_t>(nslot) &&
-                !(ok = pair_wait(bEmpty + 8 * s, ((it / nslot) - 1) & 1, abort_flag)))
+                !(ok = pair_wait_spin(bEmpty + 8 * s, ((it / nslot) - 1) & 1, abort_flag)))
               break;
             const uint32_t bar = bFull + 8 * s;
             trace(is_k ? kEvKLoad : kEvVLoad, it);
@@ -280,11 +291,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
               // S(g) = Q K_j^T (M = 256 over the pair) into S buffer g % 2, once
               // both CTAs have copied block g-2's scores out of it
               const uint32_t qb = k & 1;
-              if (j == 0 && !(ok = pair_wait(bQFull + 8 * qb, (k >> 1) & 1, abort_flag))) break;
-              if (g >= 2 && !(ok = pair_wait(bSFree + 8 * b, ((g - 2) >> 1) & 1, abort_flag))) break;
+              if (j == 0 && !(ok = pair_wait_spin(bQFull + 8 * qb, (k >> 1) & 1, abort_flag))) break;
+              if (g >= 2 && !(ok = pair_wait_spin(bSFree + 8 * b, ((g - 2) >> 1) & 1, abort_flag))) break;
               trace(kEvQkGotSFree, g);
               const uint32_t s = it % C::SK;
-              if (!(ok = pair_wait(bKFull + 8 * s, (it / C::SK) & 1, abort_flag))) break;
+              if (!(ok = pair_wait_spin(bKFull + 8 * s, (it / C::SK) & 1, abort_flag))) break;
               trace(kEvQkIssue, g);
               tc_fence_after();
               const uint32_t a_lo = q_lo0 + qb * (C::Q_BYTES >> 4);
@@ -308,21 +319,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             } else {
               // O += P(g) V_j (and the row sums) once both CTAs' codes are in TMEM
               const uint32_t s = it % C::SV;
-              if (!(ok = pair_wait(bVFull + 8 * s, (it / C::SV) & 1, abort_flag))) break;
-              if (!(ok = pair_wait(bPFull + 8 * b, (g >> 1) & 1, abort_flag))) break;
+              if (!(ok = pair_wait_spin(bVFull + 8 * s, (it / C::SV) & 1, abort_flag))) break;
+              const uint32_t pb = g % C::PB;
+              if (!(ok = pair_wait_spin(bPFull + 8 * pb, (g / C::PB) & 1, abort_flag))) break;
               trace(kEvPvGotP, g);
-              if (j == 0 && k > 0 && !(ok = pair_wait(bOEmpty, (k - 1) & 1, abort_flag))) break;
+              if (j == 0 && k > 0 && !(ok = pair_wait_spin(bOEmpty, (k - 1) & 1, abort_flag))) break;
               trace(kEvPvIssue, g);
               tc_fence_after();
               const uint32_t v_stage = sV + s * C::V_BYTES;
               const uint32_t b_lo = sdesc_lo(v_stage, sOnes - v_stage);
-              const uint32_t a_t = tmem + C::TM_P + b * C::P_COLS;
+              const uint32_t a_t = tmem + C::TM_P + pb * C::P_COLS;
 #pragma unroll
               for (int kk = 0; kk < kBN / C::MMA_K; ++kk)
                 mma_pair_ts(tmem + C::TM_O, a_t + kk * (C::MMA_K / 4), b_lo + ((kk * C::MMA_K * 64) >> 4), kSdescHi64,
                             C::IDESC_PV, (kk > 0 || j > 0) ? 1u : 0u);
-              tc_commit_pair(leader(bPDone + 8 * b));
-              tc_commit_pair(peer(bPDone + 8 * b));
+              tc_commit_pair(leader(bPDone + 8 * pb));
+              tc_commit_pair(peer(bPDone + 8 * pb));
               if (j == n - 1) {
                 tc_commit_pair(leader(bOFull + 8 * (k & 1)));
                 tc_commit_pair(peer(bOFull + 8 * (k & 1)));
@@ -335,9 +347,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         // Every MMA this thread issued has completed before either CTA frees TMEM.
         const uint32_t drain = bDrain + 8 * (warp - 1);
         tc_commit_pair(leader(drain));
-        if (!mbar_try_wait_cluster(drain, 0)) {
+        if (!mbar_try_wait(drain, 0)) {
           const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait_cluster(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+          while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
           }
         }
       }
@@ -350,7 +362,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     const int r = 32 * (warp & 3) + lane;       // row within the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint32_t tO = tmem + lane_off + C::TM_O;
-    const bool tracer = (warp & 3) == 0 && lane == 0;  // one thread per softmax group logs events
+    const bool tracer = lane == 0;  // one thread per softmax warp logs events
     uint32_t g = 0;
     bool ok = true;
 
@@ -472,16 +484,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           }
         }
 
-        // P buffer b is free once PV(g-2) has completed; O may be rescaled once
-        // PV(g-1) has (PV(g) cannot start before this group's P is in).
-        w_ok = g < 2 || pair_wait(bPDone + 8 * b, ((g >> 1) - 1) & 1, abort_flag);
+        // P buffer g % PB is free once PV(g-PB) has completed; O may be
+        // rescaled once PV(g-1) has (PV(g) cannot start before this group's P
+        // is in). Neither barrier can run a phase ahead of the one waited for:
+        // its next phase needs P of a block this group has not written yet.
+        const uint32_t pb = g % C::PB;
+        w_ok = g < static_cast<uint32_t>(C::PB) ||
+               pair_wait(bPDone + 8 * pb, ((g / C::PB) - 1) & 1, abort_flag);
         const bool resc = j > 0 && __any_sync(0xffffffffu, need);
-        if (resc) w_ok = w_ok && pair_wait(bPDone + 8 * (b ^ 1), ((g - 1) >> 1) & 1, abort_flag);
+        if (resc) w_ok = w_ok && pair_wait(bPDone + 8 * ((g - 1) % C::PB), ((g - 1) / C::PB) & 1, abort_flag);
         ok = __all_sync(0xffffffffu, w_ok);
         if (!ok) break;
         if (tracer) trace(kEvSoftmaxGotPFree, g);
         tc_fence_after();
         if (resc) {
+          if (tracer) trace(kEvRescale, g);
 #pragma unroll 1
           for (int cc = 0; cc < C::N_PV; cc += 32) {
             uint32_t orr[32];
@@ -492,10 +509,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tO + cc, orr);
           }
         }
-        tmem_st32(tmem + lane_off + C::TM_P + b * C::P_COLS, sr);
+        tmem_st32(tmem + lane_off + C::TM_P + pb * C::P_COLS, sr);
         tmem_st_wait();
         tc_fence_before();
-        warp_arrive_leader(leader(bPFull + 8 * b));
+        warp_arrive_leader(leader(bPFull + 8 * pb));
         if (tracer) trace(kEvSoftmaxPDone, g);
 
         if (j == n - 1) {

@@ -1,7 +1,8 @@
 // Per-block event trace of the attention kernels, compiled in only with
 // -DATTN_TRACE (python -m bf16_causal_prefill_fwd_b200.build --trace builds
 // lib/libb200attn_trace.so). Each record is an event id, the warp, the
-// key-block counter of the role that logged it and the SM clock (clock64), for
+// key-block counter of the role that logged it, the SM clock (clock64) and
+// %globaltimer, for
 // the first kTraceCtas CTAs of a launch; b200attn_trace_read copies them out.
 // In the normal build every trace call is empty and nothing is stored.
 //
@@ -29,6 +30,7 @@ enum TraceEvent : uint32_t {
   kEvQkGotSFree = 11,    // the QK^T issuer sees the S buffer for block g free
   kEvPvGotP = 12,        // the PV issuer sees P of block g written
   kEvSoftmaxGotPFree = 13,  // a softmax warp may write P of block g (P buffer free)
+  kEvRescale = 14,       // a softmax warp rescales O before P of block g
 };
 
 constexpr int kTraceCtas = 4;
@@ -39,6 +41,7 @@ struct TraceRec {
   uint32_t ev_warp;  // event in bits [0,8), warp in bits [8,16)
   uint32_t g;        // key-block (or ring position) counter of the logging role
   uint64_t t;        // clock64 of the SM
+  uint64_t gt;       // %globaltimer (ns; comparable across SMs)
 };
 
 #ifdef ATTN_TRACE
@@ -73,6 +76,7 @@ __device__ __forceinline__ void trace(uint32_t ev, uint32_t g) {
   r.ev_warp = ev | (w << 8);
   r.g = g;
   r.t = clock64();
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(r.gt));
   g_attn_trace[c][w][i] = r;
 }
 #else

@@ -121,15 +121,16 @@ bool regs_match(const void* kern) {
   return ok;
 }
 
-template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S>
+template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S, bool QF = false>
 int launch_attn_t(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
-  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S>;
+  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S, QF>;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, FP8, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, FP8, d_qk, p.Hkv, p.N, p.B) ||
+  // QF: the kernel reads Q itself (p.q_bf16); the Q map is encoded but unused.
+  if (!make_tmap(&tq, q, FP8 && !QF, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, FP8, d_qk, p.Hkv, p.N, p.B) ||
       !make_tmap(&tv, v, FP8, d_v, p.Hkv, p.N, p.B))
     return B200ATTN_ERR_CUDA;
-  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, FMA_P, SHARED_S>;
+  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, FMA_P, SHARED_S, QF>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
   // The kernel's role split (setmaxnreg) hands out registers from the block's
@@ -250,6 +251,17 @@ int launch_quant(const void* x, void* y, float* scale, int B, int N, int H, int 
 template <int DQK, int DV, bool HAD>
 int launch_quant_qkv(const b200::QkvQuant& a, int B, int gran, cudaStream_t stream) {
   const dim3 grid(a.H[0] + a.H[1] + a.H[2], a.nblk, B);
+  if (gran == B200ATTN_SCALE_Q_BLOCK) {
+    // Q per 128-token block: one pass (absmax and encode in one CTA per block);
+    // K and V per head: the two passes below, with no Q heads.
+    b200::QkvQuant aq = a, akv = a;
+    aq.H[1] = aq.H[2] = 0;
+    akv.H[0] = 0;
+    if (a.H[0] > 0)
+      b200::quant_qkv_encode_kernel<DQK, DV, HAD, false><<<dim3(a.H[0], a.nblk, B), b200::kQuantThreads, 0,
+                                                           stream>>>(aq);
+    return launch_quant_qkv<DQK, DV, HAD>(akv, B, B200ATTN_SCALE_PER_HEAD, stream);
+  }
   if (gran == B200ATTN_SCALE_PER_HEAD) {
     if (DQK == 128 && DV == 128 && a.H[0] % 2 == 0 && a.H[1] % 2 == 0) {
       const dim3 ggrid(grid.x / 2, a.nblk, B);
@@ -315,7 +327,8 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
   const bool fp8 = dtype == B200ATTN_FP8_E4M3;
   if (fp8) {
     if (!q_scale || !k_scale || !v_scale) return B200ATTN_ERR_INVALID;
-    if (scale_granularity != B200ATTN_SCALE_PER_HEAD && scale_granularity != B200ATTN_SCALE_PER_BLOCK)
+    if (scale_granularity != B200ATTN_SCALE_PER_HEAD && scale_granularity != B200ATTN_SCALE_PER_BLOCK &&
+        scale_granularity != B200ATTN_SCALE_Q_BLOCK)
       return B200ATTN_ERR_UNSUPPORTED;
   }
   // index arithmetic inside the kernels is 32-bit over (b, n, h) rows
@@ -324,7 +337,7 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
   const int dev_rc = device_ok(&sm_count);
   if (dev_rc != B200ATTN_OK) return dev_rc;
 
-  AttnParams p;
+  AttnParams p = {};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -336,7 +349,8 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
   if (units >= (int64_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
   p.n_units = B * Hq * p.n_pairs;
   p.causal = causal;
-  p.per_block = scale_granularity == B200ATTN_SCALE_PER_BLOCK;
+  p.per_block = fp8 && scale_granularity == B200ATTN_SCALE_PER_BLOCK;
+  p.q_per_block = fp8 && scale_granularity == B200ATTN_SCALE_Q_BLOCK;
   const double s = softmax_scale > 0.0f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d_qk));
   p.scale_log2 = static_cast<float>(s * 1.4426950408889634);
   p.q_scale = q_scale;
@@ -355,7 +369,7 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
     if (d_qk == 128) return launch_attn<128, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn<192, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
   }
-  if (!p.per_block && fp8_tile_kernel()) {
+  if (!p.per_block && !p.q_per_block && fp8_tile_kernel()) {
     if (fp8_lean_p()) {
       if (d_qk == 128) return launch_attn_tile<128, 128, true>(q, k, v, p, d_qk, d_v, sm_count, st);
       return launch_attn_tile<192, 128, true>(q, k, v, p, d_qk, d_v, sm_count, st);
@@ -363,7 +377,7 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
     if (d_qk == 128) return launch_attn_tile<128, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn_tile<192, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
   }
-  if (!p.per_block && fp8_pair_kernel()) {
+  if (!p.per_block && !p.q_per_block && fp8_pair_kernel()) {
     if (fp8_lean_p()) {
       if (d_qk == 128) return launch_attn_pair<128, 128, true>(q, k, v, p, d_qk, d_v, st);
       return launch_attn_pair<192, 128, true>(q, k, v, p, d_qk, d_v, st);
@@ -377,6 +391,56 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
   }
   if (d_qk == 128) return launch_attn<128, 128, true, false>(q, k, v, p, d_qk, d_v, sm_count, st);
   return launch_attn<192, 128, true, false>(q, k, v, p, d_qk, d_v, sm_count, st);
+}
+
+int b200attn_fwd_fp8_fused_q(const void* q, const void* k, const void* v, void* o, int B, int Hq, int Hkv, int N,
+                             int d_qk, int d_v, int causal, const float* k_scale, const float* v_scale, int hadamard,
+                             float softmax_scale, float* lse, void* q_fp8_out, float* q_scale_out, void* stream) {
+  if (!q || !k || !v || !o || !k_scale || !v_scale) return B200ATTN_ERR_INVALID;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d_qk < 1 || d_v < 1) return B200ATTN_ERR_INVALID;
+  if (Hq % Hkv != 0) return B200ATTN_ERR_INVALID;
+  if (causal != 0 && causal != 1) return B200ATTN_ERR_INVALID;
+  if (hadamard != 0 && hadamard != 1) return B200ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return B200ATTN_ERR_INVALID;
+  if (q_fp8_out && !aligned16(q_fp8_out)) return B200ATTN_ERR_INVALID;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return B200ATTN_ERR_INVALID;
+  if (q_scale_out && (reinterpret_cast<uintptr_t>(q_scale_out) & 3u)) return B200ATTN_ERR_INVALID;
+  if (!(d_v == 128 && (d_qk == 128 || d_qk == 192))) return B200ATTN_ERR_UNSUPPORTED;
+  if (!(std::isfinite(softmax_scale))) return B200ATTN_ERR_INVALID;
+  if (static_cast<int64_t>(B) * N * (Hq > Hkv ? Hq : Hkv) >= (int64_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
+  int sm_count = 0;
+  const int dev_rc = device_ok(&sm_count);
+  if (dev_rc != B200ATTN_OK) return dev_rc;
+
+  AttnParams p = {};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.G = Hq / Hkv;
+  p.n_kv = (N + b200::kBN - 1) / b200::kBN;
+  p.n_pairs = (p.n_kv + 1) / 2;
+  if (static_cast<int64_t>(B) * Hq * p.n_kv >= (int64_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
+  p.n_units = B * Hq * p.n_pairs;
+  p.causal = causal;
+  p.per_block = 0;
+  const double s = softmax_scale > 0.0f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d_qk));
+  p.scale_log2 = static_cast<float>(s * 1.4426950408889634);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.q_bf16 = static_cast<const __nv_bfloat16*>(q);
+  p.q_hadamard = hadamard;
+  p.q_codes_out = static_cast<uint8_t*>(q_fp8_out);
+  p.q_scale_out = q_scale_out;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fp8_lean_p()) {
+    if (d_qk == 128) return launch_attn_t<128, 128, true, true, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+    return launch_attn_t<192, 128, true, true, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+  }
+  if (d_qk == 128) return launch_attn_t<128, 128, true, false, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+  return launch_attn_t<192, 128, true, false, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
 }
 
 size_t b200attn_fwd_varlen_workspace_bytes(const int* cu_seqlens, int batch, int Hq) {
@@ -422,7 +486,7 @@ int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, co
   if (cudaMemcpyAsync(workspace, units.data(), need, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
 
-  AttnParams p;
+  AttnParams p = {};
   p.B = 1;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -496,9 +560,10 @@ int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale, int B, int N
 
 size_t b200attn_quantize_qkv_workspace_bytes(int B, int N, int Hq, int Hkv, int granularity) {
   if (B < 1 || N < 1 || Hq < 1 || Hkv < 1) return 0;
-  if (granularity != B200ATTN_SCALE_PER_HEAD) return 0;
+  if (granularity != B200ATTN_SCALE_PER_HEAD && granularity != B200ATTN_SCALE_Q_BLOCK) return 0;
   const size_t nblk = (static_cast<size_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
-  return static_cast<size_t>(B) * (static_cast<size_t>(Hq) + 2 * static_cast<size_t>(Hkv)) * nblk * sizeof(float);
+  const size_t heads = (granularity == B200ATTN_SCALE_PER_HEAD ? static_cast<size_t>(Hq) : 0) + 2 * static_cast<size_t>(Hkv);
+  return static_cast<size_t>(B) * heads * nblk * sizeof(float);
 }
 
 int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v, void* q_fp8, void* k_fp8, void* v_fp8,
@@ -507,7 +572,8 @@ int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v, void*
                               size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !q_fp8 || !k_fp8 || !v_fp8 || !q_scale || !k_scale || !v_scale) return B200ATTN_ERR_INVALID;
   if (B < 1 || N < 1 || Hq < 1 || Hkv < 1 || d_qk < 1 || d_v < 1) return B200ATTN_ERR_INVALID;
-  if (granularity != B200ATTN_SCALE_PER_HEAD && granularity != B200ATTN_SCALE_PER_BLOCK)
+  if (granularity != B200ATTN_SCALE_PER_HEAD && granularity != B200ATTN_SCALE_PER_BLOCK &&
+      granularity != B200ATTN_SCALE_Q_BLOCK)
     return B200ATTN_ERR_UNSUPPORTED;
   if (hadamard != 0 && hadamard != 1) return B200ATTN_ERR_INVALID;
   if (!(d_v == 128 && (d_qk == 128 || d_qk == 192))) return B200ATTN_ERR_UNSUPPORTED;
@@ -543,9 +609,10 @@ int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v, void*
   a.N = N;
   a.nblk = static_cast<int>(nblk);
   float* ws = static_cast<float*>(workspace);
-  a.partial[0] = ws;
-  a.partial[1] = ws ? ws + static_cast<size_t>(B) * Hq * nblk : nullptr;
-  a.partial[2] = ws ? ws + static_cast<size_t>(B) * (Hq + Hkv) * nblk : nullptr;
+  const size_t q_slots = granularity == B200ATTN_SCALE_PER_HEAD ? static_cast<size_t>(B) * Hq * nblk : 0;
+  a.partial[0] = granularity == B200ATTN_SCALE_PER_HEAD ? ws : nullptr;
+  a.partial[1] = ws ? ws + q_slots : nullptr;
+  a.partial[2] = ws ? ws + q_slots + static_cast<size_t>(B) * Hkv * nblk : nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d_qk == 128)
     return hadamard ? launch_quant_qkv<128, 128, true>(a, B, granularity, st)
@@ -554,6 +621,60 @@ int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v, void*
                   : launch_quant_qkv<192, 128, false>(a, B, granularity, st);
 }
 
+
+size_t b200attn_quantize_kv_workspace_bytes(int B, int N, int Hkv, int granularity) {
+  if (B < 1 || N < 1 || Hkv < 1) return 0;
+  if (granularity != B200ATTN_SCALE_PER_HEAD) return 0;
+  const size_t nblk = (static_cast<size_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  return static_cast<size_t>(B) * 2 * static_cast<size_t>(Hkv) * nblk * sizeof(float);
+}
+
+int b200attn_quantize_kv_fp8(const void* k, const void* v, void* k_fp8, void* v_fp8, float* k_scale, float* v_scale,
+                             int B, int N, int Hkv, int d_qk, int d_v, int granularity, int hadamard, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!k || !v || !k_fp8 || !v_fp8 || !k_scale || !v_scale) return B200ATTN_ERR_INVALID;
+  if (B < 1 || N < 1 || Hkv < 1 || d_qk < 1 || d_v < 1) return B200ATTN_ERR_INVALID;
+  if (granularity != B200ATTN_SCALE_PER_HEAD && granularity != B200ATTN_SCALE_PER_BLOCK)
+    return B200ATTN_ERR_UNSUPPORTED;
+  if (hadamard != 0 && hadamard != 1) return B200ATTN_ERR_INVALID;
+  if (!(d_v == 128 && (d_qk == 128 || d_qk == 192))) return B200ATTN_ERR_UNSUPPORTED;
+  const void* ptrs[4] = {k, v, k_fp8, v_fp8};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return B200ATTN_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+    return B200ATTN_ERR_INVALID;
+  const int64_t nblk = (static_cast<int64_t>(N) + b200::kQuantBlock - 1) / b200::kQuantBlock;
+  if (nblk > 65535 || 2 * static_cast<int64_t>(Hkv) > 0x7fffffff || B > 65535) return B200ATTN_ERR_UNSUPPORTED;
+  const size_t need = b200attn_quantize_kv_workspace_bytes(B, N, Hkv, granularity);
+  if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 3u)))
+    return B200ATTN_ERR_WORKSPACE;
+  int sm_count = 0;
+  const int dev_rc = device_ok(&sm_count);
+  if (dev_rc != B200ATTN_OK) return dev_rc;
+
+  // the merged Q/K/V launches with no Q heads
+  b200::QkvQuant a = {};
+  a.x[1] = static_cast<const __nv_bfloat16*>(k);
+  a.x[2] = static_cast<const __nv_bfloat16*>(v);
+  a.y[1] = static_cast<uint8_t*>(k_fp8);
+  a.y[2] = static_cast<uint8_t*>(v_fp8);
+  a.scale[1] = k_scale;
+  a.scale[2] = v_scale;
+  a.H[0] = 0;
+  a.H[1] = Hkv;
+  a.H[2] = Hkv;
+  a.N = N;
+  a.nblk = static_cast<int>(nblk);
+  float* ws = static_cast<float*>(workspace);
+  a.partial[1] = ws;
+  a.partial[2] = ws ? ws + static_cast<size_t>(B) * Hkv * nblk : nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d_qk == 128)
+    return hadamard ? launch_quant_qkv<128, 128, true>(a, B, granularity, st)
+                    : launch_quant_qkv<128, 128, false>(a, B, granularity, st);
+  return hadamard ? launch_quant_qkv<192, 128, true>(a, B, granularity, st)
+                  : launch_quant_qkv<192, 128, false>(a, B, granularity, st);
+}
 
 // ---------------------------------------------------------------------------------------------
 // Per-head quantizer without any allocation: the partial-absmax scratch lives in

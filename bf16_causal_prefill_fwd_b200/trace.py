@@ -31,8 +31,8 @@ import numpy as np
 import torch
 
 EVENTS = {1: "wait_s", 2: "have_s", 3: "max_done", 4: "p_done", 5: "qk_issue", 6: "pv_issue", 7: "k_load",
-          8: "v_load", 9: "epilogue", 10: "launch", 11: "qk_got_sfree", 12: "pv_got_p", 13: "got_pfree"}
-REC = np.dtype([("ev_warp", "<u4"), ("g", "<u4"), ("t", "<u8")])
+          8: "v_load", 9: "epilogue", 10: "launch", 11: "qk_got_sfree", 12: "pv_got_p", 13: "got_pfree", 14: "rescale"}
+REC = np.dtype([("ev_warp", "<u4"), ("g", "<u4"), ("t", "<u8"), ("gt", "<u8")])
 CAP = 12 * 4096
 CTAS = 4
 
@@ -70,6 +70,9 @@ def summarise(recs: np.ndarray) -> dict:
     out = {k: med(v) for k, v in spans.items()}
     for name in ("p_done", "qk_issue", "pv_issue", "k_load", "v_load"):
         out[f"period {name}"] = med(periods[name])
+    n_p = int(np.sum((recs["ev_warp"] & 0xFF) == 4))
+    if n_p:
+        out["rescale %"] = 100.0 * float(np.sum((recs["ev_warp"] & 0xFF) == 14)) / n_p
     launch = recs[(recs["ev_warp"] & 0xFF) == 10]
     if len(launch):
         out["grid"] = int(launch["g"][0])
@@ -98,7 +101,7 @@ def main(argv=None) -> int:
     from bf16_causal_prefill_fwd_b200.build import TRACE_LIB_PATH
 
     lib = b.load_library(a.lib or TRACE_LIB_PATH)
-    w = workloads.BY_NAME[a.workload](a.n)
+    w = workloads.sweep(a.n) if a.workload == "sweep" else workloads.BY_NAME[a.workload](a.n)
     q, k, v = (t.cuda() for t in workloads.draw(w))
     if a.dtype == "fp8":
         q8, sq, k8, sk, v8, sv = b.quantize_qkv_fp8(q, k, v)
@@ -128,7 +131,28 @@ def main(argv=None) -> int:
                                          for k, v in s.items()))
     if a.timeline:
         print_timeline(read_trace(lib, 0, reset=False), a.timeline)
+        print_pair_arrivals(read_trace(lib, 0, reset=False), read_trace(lib, 1, reset=False), a.timeline)
     return 0
+
+
+def print_pair_arrivals(r0: np.ndarray, r1: np.ndarray, nblk: int) -> None:
+    """For a few key blocks: %globaltimer (ns) at which each softmax warp of CTAs 0
+    and 1 announced P of the block, relative to the earliest."""
+    rows = []
+    for c, recs in ((0, r0), (1, r1)):
+        sel = recs[(recs["ev_warp"] & 0xFF) == 4]
+        for r in sel:
+            rows.append((int(r["g"]), c, int(r["ev_warp"]) >> 8, int(r["gt"])))
+    if not rows:
+        return
+    gmax = max(g for g, *_ in rows)
+    g0 = gmax // 4
+    print("  P announced (ns after the block's first warp), CTA.warp:")
+    for g in range(g0, g0 + nblk):
+        ev = sorted((t, c, w) for gg, c, w, t in rows if gg == g)
+        if ev:
+            t0 = ev[0][0]
+            print(f"    g={g}: " + " ".join(f"{c}.{w}:+{t - t0}" for t, c, w in ev))
 
 
 def print_timeline(recs: np.ndarray, nblk: int) -> None:
@@ -136,7 +160,8 @@ def print_timeline(recs: np.ndarray, nblk: int) -> None:
     g0 is a quarter of the way into the first unit's blocks."""
     recs = np.sort(recs, order="t")
     evs = recs["ev_warp"] & 0xFF
-    blk = recs[(evs != 7) & (evs != 8) & (evs != 10)]
+    warps = recs["ev_warp"] >> 8
+    blk = recs[(evs != 7) & (evs != 8) & (evs != 10) & np.isin(warps, [1, 2, 4, 8])]
     if not len(blk):
         return
     g0 = int(blk["g"].max()) // 4

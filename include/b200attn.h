@@ -60,7 +60,9 @@ enum { B200ATTN_BF16 = 0, B200ATTN_FP8_E4M3 = 1 };
 /* Granularity of FP8 scale factors. */
 enum {
   B200ATTN_SCALE_PER_HEAD = 0, /* one fp32 scale per (b, h): array [B, H] */
-  B200ATTN_SCALE_PER_BLOCK = 1 /* one fp32 scale per (b, h, 128-token block): [B, H, ceil(N/128)] */
+  B200ATTN_SCALE_PER_BLOCK = 1, /* one fp32 scale per (b, h, 128-token block): [B, H, ceil(N/128)] */
+  B200ATTN_SCALE_Q_BLOCK = 2    /* Q per (b, h, 128-token block) [B, Hq, ceil(N/128)]; K and V per
+                                   head [B, Hkv]: Q is quantised in one pass instead of two */
 };
 
 /*
@@ -84,8 +86,9 @@ enum {
  *        FP8 only (ignored for BF16, may be NULL): device fp32 dequantisation
  *        scales; a code c of tensor X stands for decode(c) * X_scale. Shape
  *        [B, H] for SCALE_PER_HEAD; [B, H, ceil(N/128)] for SCALE_PER_BLOCK
- *        (H = Hq for q, Hkv for k and v).
- * scale_granularity  B200ATTN_SCALE_PER_HEAD or B200ATTN_SCALE_PER_BLOCK
+ *        (H = Hq for q, Hkv for k and v); for SCALE_Q_BLOCK q's as
+ *        SCALE_PER_BLOCK, k's and v's as SCALE_PER_HEAD.
+ * scale_granularity  B200ATTN_SCALE_PER_HEAD, _PER_BLOCK or _Q_BLOCK
  * softmax_scale  s; a value <= 0 selects 1/sqrt(d_qk)
  * lse    optional (NULL allowed) fp32 [B, Hq, N]: natural-log sum over visible
  *        keys of exp(s * q.k) for each query row
@@ -102,6 +105,40 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o,
                  const float* q_scale, const float* k_scale, const float* v_scale,
                  int scale_granularity, float softmax_scale,
                  float* lse, void* stream);
+
+/*
+ * b200attn_fwd_fp8_fused_q -- the FP8 e4m3 attention of b200attn_fwd with Q
+ * given in bf16 and quantised inside the attention kernel, so that Q makes no
+ * separate pass through HBM (the quantizer then handles only K and V, e.g.
+ * with b200attn_quantize_kv_fp8).
+ *
+ * Defined by: the e4m3 inputs with absmax scale factors and the optional
+ * Hadamard rotation of Q and K ("Zyphra ZYFA: 1.76x FP8 FlashAttention
+ * Speedup on AMD MI355X", "ZYFA's performance and accuracy data"; "Zyphra 开源
+ * ZYFA …", "ZYFA 的 FP8 注意力有多准确？"). Q takes one scale per (b, h, 128-token
+ * block): the per-block granularity, with the codes and scales the quantizer
+ * gives for B200ATTN_SCALE_PER_BLOCK, bit for bit; K and V take per-head
+ * scales.
+ *
+ * q      [B, N, Hq, d_qk] bf16
+ * k, v   e4m3 codes [B, N, Hkv, d_qk] and [B, N, Hkv, d_v]
+ * k_scale, v_scale  device fp32 [B, Hkv] (per head)
+ * hadamard  1: rotate each Q row by the Hadamard transform before quantising
+ *        it (K must then have been quantised with the rotation too); 0: none
+ * q_fp8_out  optional (NULL allowed) device e4m3 [B, N, Hq, d_qk]: receives the
+ *        codes the kernel used (16-byte aligned)
+ * q_scale_out  optional (NULL allowed) device fp32 [B, Hq, ceil(N/128)]:
+ *        receives the scales the kernel used
+ * Other arguments as in b200attn_fwd (o bf16 [B, N, Hq, d_v], optional lse).
+ *
+ * Errors: INVALID (as b200attn_fwd; missing k/v scales; hadamard not 0/1;
+ * misaligned outputs), UNSUPPORTED, CUDA.
+ */
+int b200attn_fwd_fp8_fused_q(const void* q, const void* k, const void* v, void* o,
+                             int B, int Hq, int Hkv, int N, int d_qk, int d_v, int causal,
+                             const float* k_scale, const float* v_scale, int hadamard,
+                             float softmax_scale, float* lse,
+                             void* q_fp8_out, float* q_scale_out, void* stream);
 
 /*
  * b200attn_fwd_varlen_workspace_bytes -- device workspace b200attn_fwd_varlen
@@ -191,14 +228,16 @@ int b200attn_quantize_fp8(const void* x, void* x_fp8, float* scale,
 /*
  * b200attn_quantize_qkv_workspace_bytes -- device workspace
  * b200attn_quantize_qkv_fp8 needs: B*(Hq+2*Hkv)*ceil(N/128)*4 bytes for
- * SCALE_PER_HEAD, 0 for SCALE_PER_BLOCK. Returns 0 for invalid sizes.
+ * SCALE_PER_HEAD, B*2*Hkv*ceil(N/128)*4 for SCALE_Q_BLOCK (K and V only),
+ * 0 for SCALE_PER_BLOCK. Returns 0 for invalid sizes.
  */
 size_t b200attn_quantize_qkv_workspace_bytes(int B, int N, int Hq, int Hkv, int granularity);
 
 /*
  * b200attn_quantize_qkv_fp8 -- b200attn_quantize_fp8 applied to Q, K and V
  * of one attention call, in one launch per pass (two for SCALE_PER_HEAD, one
- * for SCALE_PER_BLOCK) instead of one or two per tensor. The rotation, when
+ * for SCALE_PER_BLOCK; three for SCALE_Q_BLOCK: Q's single per-block pass,
+ * then K's and V's two) instead of one or two per tensor. The rotation, when
  * hadamard == 1, applies to Q and K; V is quantised unrotated. Codes and
  * scales are bit-identical to three b200attn_quantize_fp8 calls (hadamard on
  * the first two).
@@ -221,6 +260,28 @@ int b200attn_quantize_qkv_fp8(const void* q, const void* k, const void* v,
                               int B, int N, int Hq, int Hkv, int d_qk, int d_v,
                               int granularity, int hadamard,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * b200attn_quantize_kv_workspace_bytes -- device workspace
+ * b200attn_quantize_kv_fp8 needs: B*2*Hkv*ceil(N/128)*4 bytes for
+ * SCALE_PER_HEAD, 0 for SCALE_PER_BLOCK. Returns 0 for invalid sizes.
+ */
+size_t b200attn_quantize_kv_workspace_bytes(int B, int N, int Hkv, int granularity);
+
+/*
+ * b200attn_quantize_kv_fp8 -- b200attn_quantize_qkv_fp8 for K and V only, the
+ * quantizer half of the FP8 path whose Q is quantised inside the attention
+ * kernel (b200attn_fwd_fp8_fused_q). Codes and scales are bit-identical to
+ * two b200attn_quantize_fp8 calls (hadamard on K only). Arguments as in
+ * b200attn_quantize_qkv_fp8 without the Q ones.
+ *
+ * Errors: INVALID, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+int b200attn_quantize_kv_fp8(const void* k, const void* v, void* k_fp8, void* v_fp8,
+                             float* k_scale, float* v_scale,
+                             int B, int N, int Hkv, int d_qk, int d_v,
+                             int granularity, int hadamard,
+                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * b200attn_quantize_fp8_static -- the per-head (B200ATTN_SCALE_PER_HEAD)
@@ -287,8 +348,8 @@ int b200attn_selftest_wait_timeout(int limit_us, void* stream);
  *
  * The traced build records, for the first 4 CTAs of each launch, up to 4096
  * events per warp: {uint32 event | warp << 8, uint32 block counter, uint64
- * clock64 of the SM}, 16 bytes each (event ids in csrc/attn_trace.cuh); a
- * launch overwrites the previous one's records.
+ * clock64 of the SM, uint64 %globaltimer ns}, 24 bytes each (event ids in
+ * csrc/attn_trace.cuh); a launch overwrites the previous one's records.
  * out    host buffer of cap records (may be NULL when cap == 0)
  * cta    0 .. 3
  * reset  nonzero: clear every CTA's record count afterwards

@@ -45,7 +45,7 @@ def test_max_over_ranks_with_gloo():
 
 
 class RefArgs:
-    workload, n, warmup, steps, dtype, hadamard, settle_s = "tiny", None, 3, 1, "fp8", False, 1.0
+    workload, n, warmup, steps, dtype, hadamard, settle_s, fp8_q = "tiny", None, 3, 1, "fp8", False, 1.0, "fused"
 
 
 def test_reference_arm_other_ranks_do_no_work(capsys):
@@ -68,6 +68,11 @@ def test_quantizer_summary_counts_five_bytes_per_element():
     m = bench.quantizer_summary(0.1, workloads.mla(), 6545.3)
     assert m["algorithmic_bytes"] == 5 * 16 * (192 + 192 + 128) * 16384
     assert bench.quantizer_summary(0.0, w, 6545.3) is None
+    # Q quantised inside the attention kernel: only K and V pass through the quantizer;
+    # Q per 128-token block: one pass over Q (2 bytes read, 1 written)
+    kv = 5 * (8 + 8) * 128 * 16384
+    assert bench.quantizer_summary(0.1, w, 6545.3, q_bytes=0.0)["algorithmic_bytes"] == kv
+    assert bench.quantizer_summary(0.1, w, 6545.3, q_bytes=3.0)["algorithmic_bytes"] == kv + 3 * 32 * 128 * 16384
 
 
 def test_reference_arm_line_on_rank_zero(capsys):

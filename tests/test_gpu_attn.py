@@ -176,6 +176,58 @@ def test_fp8_per_block_scales_match_oracle(shape, causal, fp8_p):
     check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
 
 
+Q_BLOCK_SHAPES = [(1, 4, 2, 300, 128), (2, 8, 2, 1000, 128), (1, 4, 4, 520, 192)]
+
+
+@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
+@pytest.mark.parametrize("shape", Q_BLOCK_SHAPES)
+@pytest.mark.parametrize("causal", [True, False])
+def test_fp8_q_block_scales_match_oracle(shape, causal, fp8_p):
+    """Q's scales per (b, h, 128-token block), K's and V's per head; Q gets very
+    different magnitudes per block so the per-block scale matters."""
+    B, Hq, Hkv, N, dqk = shape
+    q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + 11))
+    gain = torch.tensor([0.05, 3.0, 0.5, 20.0, 1.0, 0.01])[(torch.arange(N) // 128) % 6]
+    q = (q.float() * gain[None, :, None, None]).to(torch.bfloat16)
+    cq, sq = oracle.quantize_fp8(f32(q), "block", False)
+    ck, sk = oracle.quantize_fp8(f32(k), "head", False)
+    cv, sv = oracle.quantize_fp8(f32(v), "head", False)
+    q8, sq_d, k8, sk_d, v8, sv_d = to_gpu_fp8((cq, sq, ck, sk, cv, sv))
+    o, lse = b2.attn_fwd(q8, k8, v8, q_scale=sq_d, k_scale=sk_d, v_scale=sv_d, causal=causal,
+                         scale_granularity="q_block", return_lse=True)
+    assert b2.check() == 0
+    deq = (oracle.dequantize(cq, sq, "block"), oracle.dequantize(ck, sk, "head"), oracle.dequantize(cv, sv, "head"))
+    ref, ref_lse = oracle.attention(*deq, causal=causal)
+    err = oracle.rel_rms(f32(o), ref)
+    assert err <= FP8_TOL, err
+    check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
+
+
+def test_full_size_fp8_q_block_sampled():
+    """The product path with Q per block: the merged quantizer (q_block) then the
+    FP8 kernel on the full 7B-style layer; Q codes of sampled heads against the
+    oracle's per-block quantizer, output rows against fp64."""
+    w = workloads.gqa7b()
+    q, k, v = workloads.draw(w)
+    q8, sq, k8, sk, v8, sv = b2.quantize_qkv_fp8(q.cuda(), k.cuda(), v.cuda(), granularity="q_block")
+    o = b2.attn_fwd(q8, k8, v8, q_scale=sq, k_scale=sk, v_scale=sv, scale_granularity="q_block")
+    assert b2.check() == 0
+    heads, rows = sample_of(w)
+    G = w.Hq // w.Hkv
+    cq, sqr = oracle.quantize_fp8(f32(q[:, :, heads].contiguous()), "block", False)
+    assert np.array_equal(sq[:, heads].cpu().numpy(), sqr)
+    assert np.array_equal(q8.view(torch.uint8)[:, :, heads].cpu().numpy(), cq)
+    kv = [h // G for h in heads]
+    ck, skr = oracle.quantize_fp8(f32(k[:, :, kv].contiguous()), "head", False)
+    cv, svr = oracle.quantize_fp8(f32(v[:, :, kv].contiguous()), "head", False)
+    deq = (oracle.dequantize(cq, sqr, "block"), oracle.dequantize(ck, skr, "head"), oracle.dequantize(cv, svr, "head"))
+    sub = list(range(len(heads)))
+    ref8, _ = oracle_on_sample(*deq, sub, rows)
+    e = error_report(gather_sample(o, heads, rows), ref8)
+    print(f"gqa7b fp8 q_block {fmt_errors(e)}")
+    assert_within(e, FP8_TOL)
+
+
 # Per-head and per-block runs form the same e4m3 probabilities when the scales
 # agree, but may add them up in different units: with per-head scales the
 # tensor core sums the rounded probabilities in fp32, with per-block scales the
@@ -449,3 +501,21 @@ def test_sweep_fp8_error_sampled(N):
     e = error_report(got, ref8)
     print(f"sweep N={N} B={w.B} fp8 {fmt_errors(e)}; vs unquantised fp64 {oracle.rel_rms(got, ref):.2e}")
     assert_within(e, FP8_TOL)
+
+
+def test_attn_func_fp8_default_is_q_block():
+    """attn_func(fp8=True): the merged quantizer with Q per 128-token block and K, V per
+    head, then the FP8 kernel; equals calling the two directly, and matches fp64."""
+    q, k, v = workloads.draw(workloads.gaussian(1, 4, 2, 500, 128, 128, seed=27))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o = b2.attn_func(qd, kd, vd, fp8=True, hadamard=True)
+    q8, sq, k8, sk, v8, sv = b2.quantize_qkv_fp8(qd, kd, vd, granularity="q_block", hadamard=True)
+    o2 = b2.attn_fwd(q8, k8, v8, q_scale=sq, k_scale=sk, v_scale=sv, scale_granularity="q_block")
+    assert b2.check() == 0
+    assert torch.equal(o, o2)
+    cq, sqr = oracle.quantize_fp8(f32(q), "block", True)
+    ck, skr = oracle.quantize_fp8(f32(k), "head", True)
+    cv, svr = oracle.quantize_fp8(f32(v), "head", False)
+    deq = (oracle.dequantize(cq, sqr, "block"), oracle.dequantize(ck, skr, "head"), oracle.dequantize(cv, svr, "head"))
+    ref, _ = oracle.attention(*deq)
+    assert oracle.rel_rms(f32(o), ref) <= FP8_TOL

@@ -66,11 +66,12 @@ def test_full_size_single_tensor_bit_exact(name, hadamard):
 # per-head amax pass has CTAs, so each CTA loops over several.
 @pytest.mark.parametrize("shape", [(1, 300, 4, 2, 128), (2, 129, 2, 2, 192), (1, 1000, 8, 1, 128),
                                    (2, 4000, 8, 2, 128)])
-@pytest.mark.parametrize("granularity", ["head", "block"])
+@pytest.mark.parametrize("granularity", ["head", "block", "q_block"])
 @pytest.mark.parametrize("hadamard", [False, True])
 def test_qkv_in_one_launch_bit_exact(shape, granularity, hadamard):
     """Q, K and V quantised together: each tensor's codes and scales equal the
-    oracle's, with the rotation on Q and K only."""
+    oracle's, with the rotation on Q and K only ("q_block": Q per 128-token
+    block, K and V per head)."""
     B, N, Hq, Hkv, dqk = shape
     g = torch.Generator().manual_seed(B * 7 + N + Hq + dqk)
     q = (torch.randn(B, N, Hq, dqk, generator=g) * 3).to(torch.bfloat16)
@@ -78,8 +79,24 @@ def test_qkv_in_one_launch_bit_exact(shape, granularity, hadamard):
     v = torch.randn(B, N, Hkv, 128, generator=g).to(torch.bfloat16)
     outs = b2.quantize_qkv_fp8(q.cuda(), k.cuda(), v.cuda(), granularity=granularity, hadamard=hadamard)
     assert b2.check() == 0
-    for t, rot, (c, s) in ((q, hadamard, outs[0:2]), (k, hadamard, outs[2:4]), (v, False, outs[4:6])):
-        ref_codes, ref_scale = oracle.quantize_fp8(f32(t), granularity, rot)
+    for t, rot, (c, s), role in ((q, hadamard, outs[0:2], "q"), (k, hadamard, outs[2:4], "k"),
+                                 (v, False, outs[4:6], "v")):
+        gran = ("block" if role == "q" else "head") if granularity == "q_block" else granularity
+        ref_codes, ref_scale = oracle.quantize_fp8(f32(t), gran, rot)
+        assert np.array_equal(s.cpu().numpy(), ref_scale)
+        assert np.array_equal(c.view(torch.uint8).cpu().numpy(), ref_codes)
+
+
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_kv_only_quantizer_bit_exact(hadamard):
+    """b200attn_quantize_kv_fp8: K (optionally rotated) and V per head, as the oracle."""
+    g = torch.Generator().manual_seed(31)
+    k = (torch.randn(2, 700, 4, 128, generator=g) * torch.exp(torch.randn(4, 128, generator=g))).to(torch.bfloat16)
+    v = torch.randn(2, 700, 4, 128, generator=g).to(torch.bfloat16)
+    k8, sk, v8, sv = b2.quantize_kv_fp8(k.cuda(), v.cuda(), hadamard=hadamard)
+    assert b2.check() == 0
+    for t, rot, c, s in ((k, hadamard, k8, sk), (v, False, v8, sv)):
+        ref_codes, ref_scale = oracle.quantize_fp8(f32(t), "head", rot)
         assert np.array_equal(s.cpu().numpy(), ref_scale)
         assert np.array_equal(c.view(torch.uint8).cpu().numpy(), ref_codes)
 
