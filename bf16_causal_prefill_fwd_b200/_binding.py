@@ -56,10 +56,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.b200attn_quantize_qkv_fp8.restype = i
     lib.b200attn_quantize_qkv_fp8.argtypes = [vp] * 9 + [i] * 8 + [vp, sz, vp]
     lib.b200attn_fwd_varlen_workspace_bytes.restype = sz
-    lib.b200attn_fwd_varlen_workspace_bytes.argtypes = [ctypes.POINTER(ctypes.c_int), i, i]
+    lib.b200attn_fwd_varlen_workspace_bytes.argtypes = [i, i, i]
     lib.b200attn_fwd_varlen.restype = i
-    lib.b200attn_fwd_varlen.argtypes = ([vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int)] + [i] * 8
-                                        + [vp, vp, vp, f, vp, vp, sz, vp])
+    lib.b200attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, f, vp, vp, sz, vp]
     lib.b200attn_check.restype = i
     lib.b200attn_check.argtypes = [vp]
     lib.b200attn_strerror.restype = ctypes.c_char_p
@@ -184,9 +183,16 @@ def attn_fwd(q, k, v, *, causal: bool = True, softmax_scale: float | None = None
     return (out, lse) if return_lse else out
 
 
-def _cu_array(cu_seqlens):
+def _cu_device(cu_seqlens, device):
+    """cu_seqlens as a contiguous int32 tensor on `device`. A CUDA tensor is used
+    as it is (no host round trip); a list or CPU tensor is copied there, which
+    waits for the copy."""
+    if isinstance(cu_seqlens, torch.Tensor) and cu_seqlens.is_cuda:
+        if cu_seqlens.device != device or cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be int32 [batch + 1] on the device of q")
+        return cu_seqlens.contiguous()
     vals = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
-    return (ctypes.c_int * len(vals))(*vals), len(vals) - 1
+    return torch.tensor(vals, dtype=torch.int32, device=device)
 
 
 def attn_varlen_fwd(q, k, v, cu_seqlens, *, causal: bool = True, softmax_scale: float | None = None,
@@ -194,8 +200,10 @@ def attn_varlen_fwd(q, k, v, cu_seqlens, *, causal: bool = True, softmax_scale: 
                     workspace=None, stream=None):
     """Packed variable-length batch via b200attn_fwd_varlen: q [total,Hq,d_qk], k [total,Hkv,d_qk],
     v [total,Hkv,d_v] (bf16, or e4m3 with per-head fp32 scales [Hq] / [Hkv]); sequence b owns rows
-    cu_seqlens[b]:cu_seqlens[b+1] (cu_seqlens: host ints, e.g. a list or a CPU tensor). Returns
-    bf16 [total,Hq,d_v] (and fp32 lse [Hq,total] if ``return_lse``)."""
+    cu_seqlens[b]:cu_seqlens[b+1] (cu_seqlens: an int32 CUDA tensor, as flash_attn_varlen_func
+    takes it; a list or CPU tensor is copied to the device first). Returns bf16 [total,Hq,d_v]
+    (and fp32 lse [Hq,total] if ``return_lse``). The unit table is built on the device, so
+    with a CUDA cu_seqlens the call does not wait for the stream."""
     lib = load_library()
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_cuda_contig(name, t)
@@ -208,8 +216,11 @@ def attn_varlen_fwd(q, k, v, cu_seqlens, *, causal: bool = True, softmax_scale: 
     Hkv, d_v = k.shape[1], v.shape[2]
     if k.shape != (total, Hkv, d_qk) or v.shape != (total, Hkv, d_v):
         raise ValueError("shape mismatch between q, k and v")
-    cu, batch = _cu_array(cu_seqlens)
     dev = q.device
+    cu = _cu_device(cu_seqlens, dev)
+    batch = cu.numel() - 1
+    if batch < 1:
+        raise ValueError("cu_seqlens must hold batch + 1 >= 2 entries")
     if k.device != dev or v.device != dev:
         raise ValueError("q, k and v must be on one device")
     if out is None:
@@ -218,20 +229,18 @@ def attn_varlen_fwd(q, k, v, cu_seqlens, *, causal: bool = True, softmax_scale: 
         _check_buffer("out", out, (total, Hq, d_v), (torch.bfloat16,), dev)
     lse = torch.empty((Hq, total), dtype=torch.float32, device=dev) if return_lse else None
     if total == 0:  # nothing to compute (and no device memory to point at)
-        if batch < 1 or any(c != 0 for c in cu):
-            raise ValueError("cu_seqlens must be non-decreasing from 0 to total")
         return (out, lse) if return_lse else out
     if fp8:
         for name, sc, H in (("q_scale", q_scale, Hq), ("k_scale", k_scale, Hkv), ("v_scale", v_scale, Hkv)):
             if sc is None:
                 raise ValueError(f"{name} is required for e4m3 inputs")
             _check_buffer(name, sc, (H,) if sc.dim() == 1 else (1, H), (torch.float32,), dev)
-    need = int(lib.b200attn_fwd_varlen_workspace_bytes(cu, batch, Hq))
-    if workspace is None and need > 0:
+    need = int(lib.b200attn_fwd_varlen_workspace_bytes(batch, total, Hq))
+    if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = lib.b200attn_fwd_varlen(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), cu, batch, total, Hq, Hkv, d_qk, d_v, 1 if causal else 0,
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu), batch, total, Hq, Hkv, d_qk, d_v, 1 if causal else 0,
         FP8_E4M3 if fp8 else BF16, _ptr(q_scale) if fp8 else None, _ptr(k_scale) if fp8 else None,
         _ptr(v_scale) if fp8 else None, float(softmax_scale) if softmax_scale else 0.0, _ptr(lse), _ptr(workspace),
         wbytes, _stream_handle(stream))

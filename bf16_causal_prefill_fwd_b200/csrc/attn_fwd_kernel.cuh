@@ -127,6 +127,9 @@ struct AttnParams {
   // along the token dimension (B = 1, N = total tokens) and units are read from
   // this table, already ordered longest first.
   const VarlenUnit* units;
+  // Variable-length batches: the unit count, written on the device with the
+  // table (n_units is then unused).
+  const int* n_units_dev;
   // FP8 with Q quantised in the kernel (template flag QF): Q as bf16, one scale
   // per (b, h, 128-token tile) computed there, optional Hadamard rotation of
   // the rows; the codes and scales are also written out when the pointers are
@@ -327,6 +330,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int n_units = p.n_units_dev != nullptr ? *p.n_units_dev : p.n_units;
   trace_begin();
   if (threadIdx.x == 0) trace(kEvLaunch, gridDim.x);
 
@@ -401,7 +405,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool first = true, ok = true;
       for (int k = 0; ok; ++k) {
         const int u = unit_for(k, blockIdx.x, gridDim.x);
-        if (u >= p.n_units) break;
+        if (u >= n_units) break;
         const Unit x = decode_unit(u, p);
         if (is_k && !QF) {
           for (int t = 0; t < 2 && ok; ++t) {
@@ -481,7 +485,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
       for (int k = 0; ok; ++k) {
         const int u = unit_for(k, blockIdx.x, gridDim.x);
-        if (u >= p.n_units) break;
+        if (u >= n_units) break;
         const Unit x = decode_unit(u, p);
         if constexpr (C::SS) {
           // Split by role. Warp 1: S = Q_t K_j^T once the softmax has copied the
@@ -661,14 +665,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     };
     if constexpr (QF) {
       const int u0 = unit_for(0, blockIdx.x, gridDim.x);
-      if (u0 < p.n_units) {
+      if (u0 < n_units) {
         q_finish(decode_unit(u0, p), 0);
       }
     }
 
     for (int k = 0; ok; ++k) {
       const int u = unit_for(k, blockIdx.x, gridDim.x);
-      if (u >= p.n_units) break;
+      if (u >= n_units) break;
       const Unit x = decode_unit(u, p);
       const int n_t = t ? x.n1 : x.n0;
       const int q_tile = 2 * x.pair + t;
@@ -945,7 +949,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (tracer) trace(kEvSoftmaxPDone, g);
         if constexpr (QF) {
           // the next unit's Q rows travel to L2 while the epilogue waits for O
-          if (i == n_t - 1 && u_next < p.n_units) q_row_prefetch<DQK>(q_row_ptr(decode_unit(u_next, p)));
+          if (i == n_t - 1 && u_next < n_units) q_row_prefetch<DQK>(q_row_ptr(decode_unit(u_next, p)));
         }
       }
       if (!ok) break;
@@ -988,7 +992,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(bOe);
       if (tracer) trace(kEvEpilogue, g);
       if constexpr (QF) {
-        if (u_next < p.n_units) {
+        if (u_next < n_units) {
           // one Q buffer: free once this unit's last QK^T of the tile has read it
           ok = __all_sync(0xffffffffu, mbar_wait(bQEmpty + 16 * t, k & 1, abort_flag));
           if (!ok) break;

@@ -18,6 +18,7 @@
 #include "attn_fwd_pair_kernel.cuh"
 #include "attn_fwd_tile_kernel.cuh"
 #include "quant_kernel.cuh"
+#include "varlen_units.cuh"
 
 namespace {
 
@@ -281,33 +282,6 @@ int launch_quant_qkv(const b200::QkvQuant& a, int B, int gran, cudaStream_t stre
 }
 
 
-// Work units of a packed variable-length batch, longest first: one per
-// (sequence, query head, pair of 128-row query tiles). Returns false if
-// cu_seqlens is not a valid prefix-sum array ending at total.
-bool varlen_units(const int* cu, int batch, int total, int Hq, int causal, std::vector<b200::VarlenUnit>* out) {
-  if (cu[0] != 0 || cu[batch] != total) return false;
-  struct Keyed {
-    int work;
-    b200::VarlenUnit u;
-  };
-  std::vector<Keyed> units;
-  for (int b = 0; b < batch; ++b) {
-    const int len = cu[b + 1] - cu[b];
-    if (len < 0) return false;
-    const int n_kv = (len + b200::kBN - 1) / b200::kBN;
-    const int n_pairs = (n_kv + 1) / 2;
-    for (int pair = 0; pair < n_pairs; ++pair) {
-      const int work = causal ? std::min(2 * pair + 2, n_kv) : n_kv;  // key blocks of the longer tile
-      for (int h = 0; h < Hq; ++h) units.push_back({work, {cu[b], len, h, pair}});
-    }
-  }
-  std::stable_sort(units.begin(), units.end(), [](const Keyed& a, const Keyed& c) { return a.work > c.work; });
-  out->clear();
-  out->reserve(units.size());
-  for (const Keyed& k : units) out->push_back(k.u);
-  return true;
-}
-
 }  // namespace
 
 extern "C" {
@@ -443,24 +417,21 @@ int b200attn_fwd_fp8_fused_q(const void* q, const void* k, const void* v, void* 
   return launch_attn_t<192, 128, true, false, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
 }
 
-size_t b200attn_fwd_varlen_workspace_bytes(const int* cu_seqlens, int batch, int Hq) {
-  if (!cu_seqlens || batch < 1 || Hq < 1) return 0;
-  size_t units = 0;
-  for (int b = 0; b < batch; ++b) {
-    const int len = cu_seqlens[b + 1] - cu_seqlens[b];
-    if (len < 0) return 0;
-    const size_t n_kv = (static_cast<size_t>(len) + b200::kBN - 1) / b200::kBN;
-    units += (n_kv + 1) / 2 * static_cast<size_t>(Hq);
-  }
-  return units * sizeof(b200::VarlenUnit);
+size_t b200attn_fwd_varlen_workspace_bytes(int batch, int total, int Hq) {
+  if (batch < 1 || total < 0 || Hq < 1) return 0;
+  // pairs of query tiles over all sequences: sum ceil(ceil(len/128)/2) <= total/256 + batch
+  const size_t units = static_cast<size_t>(Hq) * (static_cast<size_t>(total) / (2 * b200::kBN) + batch);
+  return 16 + units * sizeof(b200::VarlenUnit);
 }
 
 int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, const int* cu_seqlens, int batch,
                         int total, int Hq, int Hkv, int d_qk, int d_v, int causal, int dtype, const float* q_scale,
                         const float* k_scale, const float* v_scale, float softmax_scale, float* lse,
                         void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q || !k || !v || !o || !cu_seqlens) return B200ATTN_ERR_INVALID;
+  if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return B200ATTN_ERR_INVALID;
   if (batch < 1 || total < 0 || Hq < 1 || Hkv < 1 || d_qk < 1 || d_v < 1) return B200ATTN_ERR_INVALID;
+  if (total == 0) return B200ATTN_OK;  // only empty sequences: nothing to read or write
+  if (!q || !k || !v || !o) return B200ATTN_ERR_INVALID;
   if (Hq % Hkv != 0) return B200ATTN_ERR_INVALID;
   if (causal != 0 && causal != 1) return B200ATTN_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return B200ATTN_ERR_INVALID;
@@ -470,21 +441,19 @@ int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, co
   if (!(std::isfinite(softmax_scale))) return B200ATTN_ERR_INVALID;
   const bool fp8 = dtype == B200ATTN_FP8_E4M3;
   if (fp8 && (!q_scale || !k_scale || !v_scale)) return B200ATTN_ERR_INVALID;
+  if (total > b200::kVarlenMaxTotal || batch > (1 << 24)) return B200ATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(total) * (Hq > Hkv ? Hq : Hkv) >= (int64_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
-  std::vector<b200::VarlenUnit> units;
-  if (!varlen_units(cu_seqlens, batch, total, Hq, causal, &units)) return B200ATTN_ERR_INVALID;
-  if (units.size() >= (size_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
-  const size_t need = units.size() * sizeof(b200::VarlenUnit);
-  if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15u)))
+  const size_t need = b200attn_fwd_varlen_workspace_bytes(batch, total, Hq);
+  if (need / sizeof(b200::VarlenUnit) >= (size_t(1) << 31)) return B200ATTN_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15u))
     return B200ATTN_ERR_WORKSPACE;
   int sm_count = 0;
   const int dev_rc = device_ok(&sm_count);
   if (dev_rc != B200ATTN_OK) return dev_rc;
-  if (units.empty()) return B200ATTN_OK;  // only empty sequences
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // pageable source: the copy is staged before cudaMemcpyAsync returns
-  if (cudaMemcpyAsync(workspace, units.data(), need, cudaMemcpyHostToDevice, st) != cudaSuccess)
-    return B200ATTN_ERR_CUDA;
+  int* ws = static_cast<int*>(workspace);
+  b200::varlen_units_kernel<<<1, b200::kVarlenBuildThreads, 0, st>>>(cu_seqlens, batch, total, Hq, causal, ws);
+  if (cudaGetLastError() != cudaSuccess) return B200ATTN_ERR_CUDA;
 
   AttnParams p = {};
   p.B = 1;
@@ -494,7 +463,7 @@ int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, co
   p.G = Hq / Hkv;
   p.n_kv = (total + b200::kBN - 1) / b200::kBN;
   p.n_pairs = (p.n_kv + 1) / 2;
-  p.n_units = static_cast<int>(units.size());
+  p.n_units = sm_count;  // the grid: the unit count itself is known on the device only
   p.causal = causal;
   p.per_block = 0;
   const double s = softmax_scale > 0.0f ? static_cast<double>(softmax_scale) : 1.0 / std::sqrt(static_cast<double>(d_qk));
@@ -504,7 +473,8 @@ int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, co
   p.v_scale = v_scale;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
-  p.units = static_cast<const b200::VarlenUnit*>(workspace);
+  p.units = reinterpret_cast<const b200::VarlenUnit*>(ws + 4);
+  p.n_units_dev = ws;
   if (!fp8) {
     if (bf16_fma_p()) {
       if (d_qk == 128) return launch_attn<128, 128, false, true>(q, k, v, p, d_qk, d_v, sm_count, st);

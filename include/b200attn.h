@@ -23,7 +23,8 @@
  *   fastest and no padding. Pointers are DEVICE pointers on the current CUDA
  *   device, 16-byte aligned, owned by the caller, and must not alias.
  * - `stream` is a cudaStream_t (NULL = the legacy default stream). All work is
- *   enqueued on it; no entry point synchronises, except b200attn_check.
+ *   enqueued on it; no entry point synchronises, except b200attn_check and
+ *   b200attn_trace_read.
  * - Return value: 0 on success, or a negative b200attn_status. On an argument
  *   error nothing is launched and no output is touched.
  * - A kernel never traps. Every wait inside a kernel is bounded (about two
@@ -142,12 +143,11 @@ int b200attn_fwd_fp8_fused_q(const void* q, const void* k, const void* v, void* 
 
 /*
  * b200attn_fwd_varlen_workspace_bytes -- device workspace b200attn_fwd_varlen
- * needs for this batch: 16 bytes per work unit, one unit per (sequence, query
- * head, pair of 128-row query tiles). cu_seqlens is the HOST array of
- * b200attn_fwd_varlen. Returns 0 for invalid arguments (and for a batch of
- * empty sequences).
+ * needs: 16 bytes of header plus 16 bytes per work unit, bounded from the
+ * sizes alone (one unit per sequence, query head and pair of 128-row query
+ * tiles: at most Hq * (total/256 + batch) units). Returns 0 for invalid sizes.
  */
-size_t b200attn_fwd_varlen_workspace_bytes(const int* cu_seqlens, int batch, int Hq);
+size_t b200attn_fwd_varlen_workspace_bytes(int batch, int total, int Hq);
 
 /*
  * b200attn_fwd_varlen -- b200attn_fwd on a batch of sequences of different
@@ -157,21 +157,28 @@ size_t b200attn_fwd_varlen_workspace_bytes(const int* cu_seqlens, int batch, int
  * q [total, Hq, d_qk], k [total, Hkv, d_qk], v [total, Hkv, d_v], o [total, Hq,
  *        d_v]: device pointers, contiguous; sequence b owns token rows
  *        [cu_seqlens[b], cu_seqlens[b+1])
- * cu_seqlens  HOST int array [batch + 1]: 0 = cu[0] <= cu[1] <= ... <=
- *        cu[batch] = total; empty sequences are allowed
+ * cu_seqlens  DEVICE int32 array [batch + 1]: 0 = cu[0] <= cu[1] <= ... <=
+ *        cu[batch] = total; empty sequences are allowed. total <= 2^21.
  * q_scale, k_scale, v_scale  FP8 only: per-head scales over the packed
  *        tensors, [Hq] and [Hkv] (b200attn_quantize_fp8 with B = 1, N = total);
  *        per-block scales are not supported here
  * lse    optional fp32 [Hq, total]
  * workspace  device memory of b200attn_fwd_varlen_workspace_bytes bytes,
- *        16-byte aligned, caller-owned; the call writes the unit table there
- *        (a host-to-device copy on `stream`) and the kernel reads it, so it
- *        must stay untouched until the kernel has finished
+ *        16-byte aligned, caller-owned, contents on entry irrelevant; a small
+ *        kernel on `stream` writes the work-unit table there from cu_seqlens,
+ *        the attention kernel then reads it, so it must stay untouched until
+ *        that kernel has finished
  * Other arguments as in b200attn_fwd. Each sequence is computed exactly as
  * b200attn_fwd computes one batch entry.
  *
- * Errors: INVALID (as b200attn_fwd, and for a cu_seqlens array that is not
- * non-decreasing from 0 to total), UNSUPPORTED, WORKSPACE, CUDA.
+ * The call reads nothing on the host and copies nothing: cu_seqlens is only
+ * read on the device, so the call returns without waiting for the stream.
+ * A cu_seqlens array that is not non-decreasing from 0 to total is found on
+ * the device: nothing is computed and the next b200attn_check returns
+ * B200ATTN_ERR_INVALID.
+ *
+ * Errors: INVALID (as b200attn_fwd; NULL or misaligned cu_seqlens),
+ * UNSUPPORTED (total above 2^21), WORKSPACE, CUDA.
  */
 int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
                         const int* cu_seqlens, int batch, int total,

@@ -146,21 +146,30 @@ def test_quantize_qkv_workspace_and_arguments_on_the_host(lib):
 
 
 def test_varlen_workspace_and_arguments_on_the_host(lib):
-    IntArr = ctypes.c_int * 4
-    cu = IntArr(0, 100, 100, 400)      # 1 + 0 + 2 pairs of 128-row tiles
-    assert lib.b200attn_fwd_varlen_workspace_bytes(cu, 3, 4) == (1 + 0 + 2) * 4 * 16
+    # bounded from the sizes: 16-byte header, then Hq * (total // 256 + batch) units of 16 bytes
+    assert lib.b200attn_fwd_varlen_workspace_bytes(3, 400, 4) == 16 + 16 * 4 * (400 // 256 + 3)
+    assert lib.b200attn_fwd_varlen_workspace_bytes(0, 400, 4) == 0
 
-    def call(cu_vals, total, ws=FAKE, wsb=1 << 20, dtype=0, q=FAKE):
-        arr = (ctypes.c_int * len(cu_vals))(*cu_vals)
-        return lib.b200attn_fwd_varlen(q, FAKE, FAKE, FAKE, arr, len(cu_vals) - 1, total, 4, 2, 128, 128, 1,
+    def call(cu=FAKE, batch=2, total=400, ws=FAKE, wsb=1 << 20, dtype=0, q=FAKE):
+        return lib.b200attn_fwd_varlen(q, FAKE, FAKE, FAKE, cu, batch, total, 4, 2, 128, 128, 1,
                                        dtype, None, None, None, 0.0, None, ws, wsb, None)
-    assert call([0, 100, 50, 400], 400) == -1        # decreasing
-    assert call([1, 100, 400], 400) == -1            # not starting at 0
-    assert call([0, 100, 399], 400) == -1            # not ending at total
-    assert call([0, 100, 400], 400, q=None) == -1
-    assert call([0, 100, 400], 400, dtype=1) == -1   # FP8 without scales
-    assert call([0, 100, 400], 400, ws=None) == -5
-    assert call([0, 100, 400], 400, wsb=16) == -5
+    # cu_seqlens is read on the device only; what the host can check it checks
+    assert call(cu=None) == -1
+    assert call(cu=FAKE + 2) == -1                   # misaligned int array
+    assert call(batch=0) == -1
+    assert call(q=None) == -1
+    assert call(dtype=1) == -1                       # FP8 without scales
+    assert call(ws=None) == -5
+    assert call(wsb=16) == -5
+    assert call(total=(1 << 21) + 1) == -2           # above the device-side unit builder's limit
+    assert call(total=0, q=None) == 0                # only empty sequences: nothing to do
+
+
+def test_q_block_granularity_on_the_host(lib):
+    # Q per 128-token block needs no partial absmax: only K's and V's
+    assert lib.b200attn_quantize_qkv_workspace_bytes(2, 300, 4, 2, 2) == 2 * (2 * 2) * 3 * 4
+    assert qkv(lib, gran=2, wsb=8) == -5
+    assert fwd(lib, dtype=1, qs=FAKE, ks=FAKE, vs=FAKE, gran=3) == -2
 
 
 def header_prototypes():
@@ -183,7 +192,7 @@ def ctype_of(c):
         base = c.replace("const", "").replace("*", "").strip()
         if base == "char":
             return ctypes.c_char_p
-        return ctypes.POINTER(ctypes.c_int) if base == "int" else ctypes.c_void_p
+        return ctypes.c_void_p  # every pointer argument is a device (or caller-owned) address
     return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t}[c]
 
 

@@ -1,6 +1,8 @@
 """Packed variable-length batches (b200attn_fwd_varlen) against the fp64 oracle,
 sequence by sequence. Each sequence must come out as b200attn_fwd computes one
 batch entry: the same parity bounds, and for BF16 the same bytes."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -91,3 +93,55 @@ def test_varlen_func_fp8_path_and_empty_batch():
     assert oracle.rel_rms(f32(o), ref) <= 0.1  # against unquantised inputs: input rounding included
     z = torch.empty((0, 4, 128), dtype=torch.bfloat16, device="cuda")
     assert b2.attn_varlen_fwd(z, z[:, :2], z[:, :2], [0, 0]).shape == (0, 4, 128)
+
+
+def test_varlen_call_does_not_wait_for_the_stream():
+    """With cu_seqlens in device memory the call reads nothing on the host: it
+    returns while a long kernel queued before it is still running, and the
+    result is the one a call on an idle stream gives."""
+    q, k, v, cu = packed([300, 0, 1000, 129], 4, 2, 128, seed=41)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    cu_d = torch.from_numpy(cu).cuda()
+    ref = b2.attn_varlen_fwd(qd, kd, vd, cu_d)
+    out = torch.empty_like(ref)
+    ws = torch.empty(b2.load_library().b200attn_fwd_varlen_workspace_bytes(len(cu) - 1, int(cu[-1]), 4),
+                     dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    busy = torch.cuda.Event()
+    torch.cuda._sleep(2_000_000_000)   # about a second of spinning on the current stream
+    busy.record()
+    t0 = time.perf_counter()
+    b2.attn_varlen_fwd(qd, kd, vd, cu_d, out=out, workspace=ws)
+    dt = time.perf_counter() - t0
+    still_busy = not busy.query()
+    assert b2.check() == 0
+    assert still_busy and dt < 0.1, (still_busy, dt)
+    assert torch.equal(out, ref)
+
+
+def test_varlen_invalid_cu_seqlens_reported_on_the_device():
+    """A cu_seqlens that does not run from 0 to total is found by the unit builder:
+    nothing is computed, b200attn_check reports INVALID, and later calls work."""
+    q, k, v, cu = packed([300, 129], 4, 2, 128, seed=42)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    bad = torch.tensor([0, 500, 429], dtype=torch.int32, device="cuda")   # decreasing step
+    out = torch.full((429, 4, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    b2.attn_varlen_fwd(qd, kd, vd, bad, out=out)
+    assert b2.check() == -1
+    assert bool((out == 7.0).all())
+    o = b2.attn_varlen_fwd(qd, kd, vd, torch.from_numpy(cu).cuda())
+    assert b2.check() == 0
+    ref, _ = oracle_per_sequence(f32(q), f32(k), f32(v), cu, True)
+    assert oracle.rel_rms(f32(o), ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_skewed_lengths(causal):
+    """One long sequence among many short ones (the unit table groups them by
+    work): every sequence against the oracle."""
+    lengths = [4096] + [130, 1, 257, 64, 0, 512, 33] * 3
+    q, k, v, cu = packed(lengths, 8, 2, 128, seed=43)
+    o = b2.attn_varlen_fwd(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cu).cuda(), causal=causal)
+    assert b2.check() == 0
+    ref, _ = oracle_per_sequence(f32(q), f32(k), f32(v), cu, causal)
+    assert oracle.rel_rms(f32(o), ref) <= BF16_TOL
