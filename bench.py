@@ -92,7 +92,8 @@ def load_peaks():
 
 def kernel_sources_sha() -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd_kernel.cuh", "attn_fwd_pair_kernel.cuh", "attn_fwd_tile_kernel.cuh", "sm100_ptx.cuh"):
+    for f in ("attn_fwd_kernel.cuh", "attn_fwd_pair_kernel.cuh", "attn_fwd_tile_kernel.cuh", "sm100_ptx.cuh",
+              "q_encode.cuh", "attn_trace.cuh"):
         with open(os.path.join(ROOT, "bf16_causal_prefill_fwd_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -282,26 +283,19 @@ def head_flops(w: workloads.Workload) -> float:
     return float(w.N) * w.N * (w.d_qk + w.d_v)
 
 
-def cpu_baseline(q, k, v, w: workloads.Workload, full_limit_s: float = 45.0) -> dict:
-    """The oracle, as it stands, on the host cores. One query head is timed first;
-    if the whole workload (every batch entry and head) is then expected to take at
-    most full_limit_s, the whole workload is run and timed in one call."""
-    import oracle
-    t_head = oracle_heads(q, k, v, w, [0])
-    n_heads = w.B * w.Hq
-    cores = len(os.sched_getaffinity(0))
-    if t_head * n_heads <= full_limit_s:
-        to64 = lambda t: t.float().numpy().astype(np.float64)
-        q64, k64, v64 = to64(q), to64(k), to64(v)
-        t0 = time.perf_counter()
-        oracle.attention(q64, k64, v64, causal=True)
-        secs = time.perf_counter() - t0
-        return {"value": w.flops / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                "sample": f"the whole workload ({w.B} x {w.Hq} heads x {w.N} rows), fp64, one call",
-                "seconds": secs}
-    return {"value": head_flops(w) / t_head / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"every row of query head 0 of batch 0 (1/{n_heads} of the workload), fp64",
-            "seconds": t_head}
+def cpu_baseline(q, k, v, w: workloads.Workload, n_heads: int = 8) -> dict:
+    """The oracle, as it stands, on the host cores: every row of n_heads query heads of
+    batch entry 0, spread over the heads (one per key/value head on the GQA layers), each
+    head run as its own problem. A bounded sample: the whole 7B-style layer, run once
+    through the oracle in one call, took 116 s on the 16 host cores of the GPU machine."""
+    step = max(1, w.Hq // n_heads)
+    heads = list(range(0, w.Hq, step))[:n_heads]
+    secs = sum(oracle_heads(q, k, v, w, [h]) for h in heads)
+    return {"value": len(heads) * head_flops(w) / secs / 1e12, "unit": "TFLOP/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"every row of query heads {heads} of batch 0 ({len(heads)}/{w.B * w.Hq} of the workload), "
+                      f"fp64, one oracle call per head",
+            "seconds": secs}
 
 
 def run_reference(args, rank: int, world: int):
@@ -380,9 +374,9 @@ class Path:
             self.sv = torch.empty((B, Hkv), dtype=torch.float32, device=dev)
             ws = max(b2.quantize_qkv_workspace_bytes(B, N, Hq, Hkv, self.gran), 4)
             self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
-        # FP8: absmax and encode passes over K and V (with Q too when not fused; one
-        # launch each), attention
-        self.launches_per_step = 3 if dtype == "fp8" else 1
+        # FP8: absmax and encode passes over K and V (and Q with per-head scales; one
+        # launch each), Q's single pass with per-block scales, attention
+        self.launches_per_step = (4 if fp8_q == "qblock" else 3) if dtype == "fp8" else 1
 
     def step(self, ev_a0=None, ev_a1=None):
         b2 = self.b2
@@ -544,6 +538,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "kernel": kernel_key, "kernel_ms": ams,
                 "peak_source": fp8_peak_src if dtype == "fp8" else f"{peak_src} bf16 burst {bf16_peak} TFLOP/s",
                 "frac_of_spec_dense": achieved / (4500.0 if dtype == "fp8" else 2250.0)}
+        if dtype == "fp8":  # against the bf16 peak times the nominal e4m3/bf16 ratio, for comparison
+            roof["frac_of_bf16_peak_x2"] = achieved / (2.0 * bf16_peak)
         quant = None
         if dtype == "fp8":
             qms = max_over_ranks(statistics.mean([s - a for s, a in zip(step_ms, attn_ms)]), dist_on)

@@ -53,25 +53,6 @@ __device__ __forceinline__ void bf16x8_to_float(const uint4& raw, float (&v)[8])
   }
 }
 
-// Load the 8 (or 4) elements this lane holds of one row; `row` is clamped by the caller.
-template <int D>
-__device__ __forceinline__ void load_lane(const __nv_bfloat16* row, int lane, float (&v)[8]) {
-  if constexpr (D == 128) {
-    bf16x8_to_float(*reinterpret_cast<const uint4*>(row + 8 * (lane & 15)), v);
-  } else {
-    if (lane < 16) {
-      bf16x8_to_float(*reinterpret_cast<const uint4*>(row + 8 * lane), v);
-    } else {
-      const uint2 raw = *reinterpret_cast<const uint2*>(row + 128 + 4 * (lane - 16));
-      v[0] = __uint_as_float(raw.x << 16);
-      v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-      v[2] = __uint_as_float(raw.y << 16);
-      v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-      v[4] = v[5] = v[6] = v[7] = 0.0f;
-    }
-  }
-}
-
 // In-place normalised Walsh-Hadamard transform of this lane's segment. Lanes
 // 0-15 (and, for d = 128, lanes 16-31) hold 8 consecutive elements of a
 // 128-wide row; for d = 192 lanes 16-31 hold 4 consecutive elements of the
@@ -108,25 +89,53 @@ __device__ __forceinline__ void rotate_lane(int lane, float (&v)[8]) {
   for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], c);
 }
 
+// The raw bf16 words this lane holds of one row: 8 elements (uint4), or 4 on
+// the 64-wide tail lanes of a 192-wide row (.x, .y).
+template <int D>
+__device__ __forceinline__ uint4 load_lane_raw(const __nv_bfloat16* row, int lane) {
+  if (D == 128 || lane < 16) return *reinterpret_cast<const uint4*>(row + 8 * (lane & 15));
+  const uint2 r = *reinterpret_cast<const uint2*>(row + 128 + 4 * (lane - 16));
+  return make_uint4(r.x, r.y, 0u, 0u);
+}
+
+// The lane's values of one row from its raw words (rotated when HAD): lanes
+// 0-15 (all lanes for d = 128) hold 8 consecutive elements of a 128-wide row,
+// for d = 192 lanes 16-31 hold 4 of the 64-wide tail (the other 4 are zero).
+template <int D, bool HAD>
+__device__ __forceinline__ void lane_values(const uint4& raw, int lane, float (&v)[8]) {
+  bf16x8_to_float(raw, v);  // the tail lanes' zero words give zeros
+  if constexpr (HAD) rotate_lane<D>(lane, v);
+}
+
+// One 128-token block of (b, h): the raw words stay in registers (half the
+// registers of fp32 values, so two CTAs fit on an SM at d = 192) and the
+// values are formed again where they are needed.
 template <int D, bool HAD>
 __device__ __forceinline__ void load_block(const __nv_bfloat16* __restrict__ x, int b, int h, int blk, int N, int H,
-                                           int warp, int lane, float (&v)[QuantLayout<D>::ITERS][8], float& amax) {
+                                           int warp, int lane, uint4 (&raw)[QuantLayout<D>::ITERS], float& amax) {
   using L = QuantLayout<D>;
   const int sub = (D == 128) ? (lane >> 4) : 0;
 #pragma unroll
   for (int it = 0; it < L::ITERS; ++it) {
     const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
     const int rc = row < N ? row : N - 1;
-    load_lane<D>(x + (static_cast<size_t>(b) * N + rc) * H * D + static_cast<size_t>(h) * D, lane, v[it]);
+    raw[it] = load_lane_raw<D>(x + (static_cast<size_t>(b) * N + rc) * H * D + static_cast<size_t>(h) * D, lane);
   }
+  // every load of the block is issued before the first value is used (measured:
+  // without this the d = 192 absmax pass interleaved loads and maxima and
+  // reached 1.7 TB/s)
+#pragma unroll
+  for (int it = 0; it < L::ITERS; ++it)
+    asm volatile("" : "+r"(raw[it].x), "+r"(raw[it].y), "+r"(raw[it].z), "+r"(raw[it].w));
   amax = 0.0f;
 #pragma unroll
   for (int it = 0; it < L::ITERS; ++it) {
-    if constexpr (HAD) rotate_lane<D>(lane, v[it]);
+    float v[8];
+    lane_values<D, HAD>(raw[it], lane, v);
     const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
     if (row < N) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[it][e]));
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
     }
   }
 }
@@ -149,9 +158,9 @@ template <int D, bool HAD>
 __device__ __forceinline__ void absmax_body(const __nv_bfloat16* __restrict__ x, float* __restrict__ partial, int N,
                                             int H, int nblk, int blk, int h, int b, float* red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float v[QuantLayout<D>::ITERS][8];
+  uint4 raw[QuantLayout<D>::ITERS];
   float m;
-  load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, v, m);
+  load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, raw, m);
   m = block_max(m, red);
   if (threadIdx.x == 0) partial[(static_cast<size_t>(b) * H + h) * nblk + blk] = m;
 }
@@ -164,9 +173,9 @@ __device__ __forceinline__ void encode_body(const __nv_bfloat16* __restrict__ x,
                                             int H, int nblk, int blk, int h, int b, float* red) {
   using L = QuantLayout<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float v[L::ITERS][8];
+  uint4 raw[L::ITERS];
   float m;
-  load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, v, m);
+  load_block<D, HAD>(x, b, h, blk, N, H, warp, lane, raw, m);
   if constexpr (PER_HEAD) {
     m = 0.0f;
     const float* ph = partial + (static_cast<size_t>(b) * H + h) * nblk;
@@ -189,10 +198,12 @@ __device__ __forceinline__ void encode_body(const __nv_bfloat16* __restrict__ x,
     const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
     if (row < N) {
       uint8_t* dst = y + (static_cast<size_t>(b) * N + row) * H * D + static_cast<size_t>(h) * D;
+      float v[8];
+      lane_values<D, HAD>(raw[it], lane, v);
       uint32_t c[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        c[q] = pack_e4m3x2(__fmul_rn(v[it][2 * q], inv), __fmul_rn(v[it][2 * q + 1], inv));
+        c[q] = pack_e4m3x2(__fmul_rn(v[2 * q], inv), __fmul_rn(v[2 * q + 1], inv));
       if (D == 128 || lane < 16) {
         *reinterpret_cast<uint2*>(dst + 8 * (lane & 15)) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
       } else {
