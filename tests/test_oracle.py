@@ -345,6 +345,20 @@ def test_quantize_per_block_scales():
         np.testing.assert_array_equal(scales[:, :, blk], amax / np.float32(448))
     dq = oracle.dequantize(codes, scales, "block")
     assert oracle.rel_rms(dq, x) < 0.04
+    # element by element, as for per-head scales: e4m3 RNE is within 2^-4 relative in the
+    # normal range and 2^-10 of the block's scale below it (half the subnormal spacing 2^-9)
+    scale_tok = np.repeat(scales, 128, axis=2)[:, :, :300].transpose(0, 2, 1)[..., None]   # [B, N, H, 1]
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, scale_tok * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(dq - x) <= bound)
+    # each block's largest magnitude is exactly +-448 (code 0x7E / 0xFE)
+    for blk, sl in enumerate([slice(0, 128), slice(128, 256), slice(256, 300)]):
+        for h in range(2):
+            flat = np.abs(x[0, sl, h]).ravel()
+            assert codes[0, sl, h].ravel()[np.argmax(flat)] & 0x7F == 0x7E
+    # a plausible slip -- block 1 encoded with block 0's scale -- breaks the bound
+    wrong = codes.copy()
+    wrong[:, 128:256, 0] = oracle.e4m3_encode((x[:, 128:256, 0] / scales[0, 0, 0]).astype(np.float32))
+    assert not np.all(np.abs(oracle.dequantize(wrong, scales, "block") - x) <= bound)
 
 
 def test_quantize_zero_tensor():
