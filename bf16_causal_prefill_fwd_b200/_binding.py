@@ -36,11 +36,12 @@ class B200AttnError(RuntimeError):
 
 def load_library(path: str | None = None) -> ctypes.CDLL:
     """Load libb200attn.so (raises if it is missing: build it with
-    ``python -m bf16_causal_prefill_fwd_b200.build``)."""
+    ``python -m bf16_causal_prefill_fwd_b200.build``). B200ATTN_LIBRARY, when set,
+    names another build of the same library to load instead (A/B runs)."""
     global _lib
     if _lib is not None:
         return _lib
-    path = path or LIB_PATH
+    path = path or os.environ.get("B200ATTN_LIBRARY") or LIB_PATH
     if not os.path.exists(path):
         raise RuntimeError(f"{path} is missing; build it with `python -m bf16_causal_prefill_fwd_b200.build`")
     lib = ctypes.CDLL(path)

@@ -285,6 +285,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort_flag);
 }
 
+// For roles whose waits are not on the critical path (the TMA producers, whose
+// rings run several blocks ahead): sleep between polls so that the spinning
+// thread gives its issue slots to the softmax warps of its SM sub-partition.
+__device__ __forceinline__ bool mbar_wait_lazy(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicCAS(&g_b200attn_status, 0, kStatusTimeout);
+      return false;
+    }
+    __nanosleep(256);
+  }
+  return true;
+}
+
 template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S, bool QF = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -410,7 +427,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (is_k && !QF) {
           for (int t = 0; t < 2 && ok; ++t) {
             if (!first) {
-              ok = mbar_wait(bQEmpty + 16 * t, qe_par[t], abort_flag);
+              ok = mbar_wait_lazy(bQEmpty + 16 * t, qe_par[t], abort_flag);
               qe_par[t] ^= 1;
               if (!ok) break;
             }
@@ -424,7 +441,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         for (int j = 0; j < x.n1 && ok; ++j, ++it) {
           const uint32_t s = it % nslot;
-          if (it >= static_cast<uint32_t>(nslot) && !(ok = mbar_wait(bEmpty + 8 * s, ((it / nslot) - 1) & 1, abort_flag)))
+          if (it >= static_cast<uint32_t>(nslot) && !(ok = mbar_wait_lazy(bEmpty + 8 * s, ((it / nslot) - 1) & 1, abort_flag)))
             break;
           const uint32_t bar = bFull + 8 * s;
           trace(is_k ? kEvKLoad : kEvVLoad, it);
@@ -900,6 +917,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             w_ok = w_ok && mbar_wait(bPDone + 8 * (t * C::PBX + (g - 1) % C::PB), ((g - 1) / C::PB) & 1, abort_flag);
           ok = __all_sync(0xffffffffu, w_ok);
           if (!ok) break;
+          if (tracer) trace(kEvSoftmaxGotPFree, g);
           tc_fence_after();
           if (resc) {
 #pragma unroll 1

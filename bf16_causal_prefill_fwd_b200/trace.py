@@ -66,6 +66,10 @@ def summarise(recs: np.ndarray) -> dict:
             spans["max"].append(e["max_done"] - e["have_s"])
         if "max_done" in e and "p_done" in e:
             spans["P"].append(e["p_done"] - e["max_done"])
+        if "max_done" in e and "got_pfree" in e:
+            spans["P codes + buffer wait"].append(e["got_pfree"] - e["max_done"])
+        if "got_pfree" in e and "p_done" in e:
+            spans["P store"].append(e["p_done"] - e["got_pfree"])
     med = lambda v: float(statistics.median(v)) if v else float("nan")
     out = {k: med(v) for k, v in spans.items()}
     for name in ("p_done", "qk_issue", "pv_issue", "k_load", "v_load"):
