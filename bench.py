@@ -60,8 +60,9 @@ def parse_args():
                     help="FP8 step: Q quantised inside the attention kernel (fused, per 128-token tile), by the "
                          "quantizer per head (separate), or by the quantizer per 128-token block in one pass "
                          "(qblock); K and V per head by the quantizer")
-    ap.add_argument("--fp8-p", choices=["lean", "mufu"], default=None,
-                    help="how the FP8 kernel forms probabilities (default: the library default, Lean P)")
+    ap.add_argument("--fp8-p", choices=["lean", "mufu", "block"], default=None,
+                    help="how the FP8 kernel forms probabilities (default: the library default, Lean P; block = "
+                         "Lean P with one power-of-two scale per 64-key half block, applied by the block-scaled MMA)")
     ap.add_argument("--settle-s", type=float, default=1.0,
                     help="untimed back-to-back steps before timing so clocks reach their sustained level")
     ap.add_argument("--no-e2e", action="store_true")
@@ -492,17 +493,20 @@ def max_over_ranks(x: float, dist_on: bool, device: str = "cuda") -> float:
 
 def kernel_name(dtype: str, w: workloads.Workload, fused_q: bool = False) -> str:
     """The attention kernel (and probability mode) the library runs for this call."""
+    env_p = os.environ.get("B200ATTN_FP8_P")
     if dtype == "fp8" and fused_q:
-        fp8_p = "mufu" if os.environ.get("B200ATTN_FP8_P") == "mufu" else "lean"
+        fp8_p = "mufu" if env_p == "mufu" else "lean"
         return f"attn_fwd_kernel<{w.d_qk},{w.d_v},fp8,{fp8_p},fused-q>"
     if dtype == "fp8":
-        fp8_p = "mufu" if os.environ.get("B200ATTN_FP8_P") == "mufu" else "lean"
+        fp8_p = "mufu" if env_p == "mufu" else "lean"
         if os.environ.get("B200ATTN_FP8_TILE") == "1":
             kname = "attn_fwd_tile_kernel"
         elif os.environ.get("B200ATTN_FP8_PAIR") == "1":
             kname = "attn_fwd_pair_kernel"
         else:
             kname = "attn_fwd_kernel"
+            if env_p == "block" and os.environ.get("B200ATTN_SHARED_S") != "0":
+                fp8_p = "lean,block-scaled"
         return f"{kname}<{w.d_qk},{w.d_v},fp8,{fp8_p}>"
     bf16_p = "mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed"
     return f"attn_fwd_kernel<{w.d_qk},{w.d_v},bf16,{bf16_p}>"

@@ -69,10 +69,12 @@
 //  * Lean P ("ZYFA 如何工作？", Lean P：用一次乘加代替指数运算): read as an
 //    integer, the e4m3 code of 2^x is close to 8x + 56 (+8 per doubling), so the
 //    code is built with fused multiply-adds and no exponential: one packed FFMA
-//    gives w = (8x + 56)/126 for two scores, a convert to f16x2 clamps negative
-//    w to 0 (w <= 120/126 by the choice of T and E), and one f16x2 FMA with the
-//    magic 1536 (f16 spacing 1 in [1024, 2048)) leaves round(126 w) in the low
-//    byte of each lane; one PRMT gathers four codes.
+//    gives v = 8x + 56 + 1536 for two scores, one convert to f16x2 rounds v to
+//    an integer (f16 spacing is 1 in [1024, 2048)), so the low byte of each
+//    lane is round(8x + 56) (<= 120 by the choice of T and E), one f16x2 max
+//    against 1536 clamps negative codes to 0, and one PRMT gathers four codes.
+//    The fp32 value is rounded once; rounding it to f16 first and scaling it
+//    after (double rounding) moves about one code in a hundred by one step.
 // Either way l is the sum of the rounded probabilities the PV MMA multiplies
 // ("逐块缩放与舍入行和": divide by the sum of the rounded probabilities): the
 // bits (code << 7) read as an f16 are exactly decode(code) / 256 for every
@@ -140,7 +142,7 @@ struct AttnParams {
   float* q_scale_out;
 };
 
-template <int DQK, int DV, bool FP8, bool FMA_P = false, bool SHARED_S = true, bool QF = false>
+template <int DQK, int DV, bool FP8, bool FMA_P = false, bool SHARED_S = true, bool QF = false, bool BSP = false>
 struct AttnCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int CHUNK_ELEMS = 128 / ESZ;  // elements in one 128-byte swizzled row
@@ -183,10 +185,25 @@ struct AttnCfg {
   static constexpr int NUM_BARS = 4 + 4 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
   static constexpr int SMEM_BYTES = 2 * Q_BUFS * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES +
                                     1024 /*bars*/ + 1024 /*align*/;
-  static constexpr float T_LAG = FP8 ? 4.0f : 8.0f;   // allowed lag of the running max (log2)
+  // BS: block-scaled P. Every 64-key half of a block carries its own power-of-two
+  // scale, applied by the tensor core (kind::mxf8f6f4.block_scale): the codes of
+  // a half are formed with its largest probability in the top binade, and the
+  // half's UE8M0 scale factor undoes the shift. The scale factors of tile t sit
+  // in the spare columns of O_t: 4 columns for A (row m at column m / 32), then
+  // 12 columns of B scales, all 1.0.
+  static constexpr bool BS = BSP && RS;
+  static constexpr int SF_COL = DVX;                 // A scales, from the start of O_t
+  static constexpr int SFB_COL = DVX + 4;            // B scales
+  static constexpr int SFB_COLS = O_STRIDE - SFB_COL;
+  // Allowed lag of the running max (log2). With one scale per block P stays
+  // within e4m3's range whatever the lag, so BS may lag as far as BF16.
+  static constexpr float T_LAG = FP8 && !BS ? 4.0f : 8.0f;
   static constexpr float E_SHIFT = FP8 ? 4.0f : 0.0f;  // exponent shift of P (log2); max P = 2^8
   static constexpr uint32_t IDESC_QK = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, kBN, false);
-  static constexpr uint32_t IDESC_PV = idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DVX, true);
+  static constexpr uint32_t IDESC_PV =
+      BS ? idesc_block_scaled(kBM, DVX, true) : idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DVX, true);
+  static_assert(!BSP || (FP8 && FMA_P && RS), "block-scaled P is a variant of Lean P with tensor-core row sums");
+  static_assert(!BS || SFB_COLS >= 8, "B scales need the columns n / 32 of N = d_v + 16");
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
   static_assert(SK >= 2 && SV >= 1, "K/V rings");
   static_assert(!SS || TM_P + 2 * PB * P_COLS <= 512, "TMEM budget");
@@ -302,11 +319,11 @@ __device__ __forceinline__ bool mbar_wait_lazy(uint32_t bar, uint32_t parity, vo
   return true;
 }
 
-template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S, bool QF = false>
+template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S, bool QF = false, bool BSP = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S, QF>;
+  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S, QF, BSP>;
   static_assert(!QF || (FP8 && SHARED_S), "Q is quantised in the kernel only on the FP8 shared-S path");
   extern __shared__ uint8_t smem_raw[];
 
@@ -487,10 +504,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t b_lo = C::RS ? sdesc_lo(v_stage, sOnes - v_stage) : v_lo0 + s * (C::V_BYTES >> 4);
         const uint32_t a_t = tmem + (C::SS ? C::TM_P + pbuf * C::P_COLS : t * 128);
         const uint32_t acc = accumulate ? 1u : 0u;
+        if constexpr (C::BS) {
+          // K step kk covers keys 32 kk .. 32 kk + 31 and reads scale byte kk of each row
 #pragma unroll
-        for (int kk = 0; kk < kBN / C::MMA_K; ++kk)
-          mma_ts_lo<FP8>(d, a_t + kk * (C::MMA_K * C::ESZ / 4), b_lo + ((kk * C::MMA_K * 128) >> 4), C::IDESC_PV,
-                         kk > 0 ? 1u : acc);
+          for (int kk = 0; kk < kBN / C::MMA_K; ++kk)
+            mma_ts_bs_lo(d, a_t + kk * (C::MMA_K / 4), b_lo + ((kk * C::MMA_K * 128) >> 4), C::IDESC_PV,
+                         d + C::SF_COL, d + C::SFB_COL, static_cast<uint32_t>(kk), kk > 0 ? 1u : acc);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kBN / C::MMA_K; ++kk)
+            mma_ts_lo<FP8>(d, a_t + kk * (C::MMA_K * C::ESZ / 4), b_lo + ((kk * C::MMA_K * 128) >> 4), C::IDESC_PV,
+                           kk > 0 ? 1u : acc);
+        }
       };
       uint32_t kit = 0, vit = 0;  // K and V ring positions
       uint32_t nq = 0;            // QK^T products issued (SS: uses of the one S buffer)
@@ -632,6 +657,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tP = tmem + lane_off + C::TM_P + t * C::PB * C::P_COLS;  // SS
     const uint32_t bS = bSFull + 8 * t;
     const uint32_t bOf = bOFull + 8 * t, bOe = bOEmpty + 8 * t;
+    if constexpr (C::BS) {
+      // B scales 1.0 (UE8M0 127) in this warp's lanes; the first P handoff's
+      // store wait covers these stores too.
+#pragma unroll
+      for (int c = 0; c < C::SFB_COLS; c += 4) tmem_st4_same(tO + C::SFB_COL + c, 0x7F7F7F7Fu);
+    }
     uint32_t s_par = 0, o_par = 0;
     uint32_t g = 0;  // key blocks this warpgroup has finished (SS buffer and parity index)
     const bool tracer = (warp & 3) == 0 && lane == 0;  // one thread per softmax warpgroup logs events
@@ -703,12 +734,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // far in this unit and O is kept in units of s_ref (rescaled when it grows).
       float c_log2 = p.scale_log2;
       float v_mult = 1.0f;
+      float sq_blk = 1.0f;  // per-block scales: this tile's Q scale
       const float* ks_blk = nullptr;
       const float* vs_blk = nullptr;
       if constexpr (FP8) {
         if (p.per_block) {
           const size_t kv_row = static_cast<size_t>(x.b * p.Hkv + x.hkv) * p.n_kv;
-          c_log2 *= __ldg(p.q_scale + static_cast<size_t>(x.b * p.Hq + x.hq) * p.n_kv + q_tile);
+          sq_blk = __ldg(p.q_scale + static_cast<size_t>(x.b * p.Hq + x.hq) * p.n_kv + q_tile);
           ks_blk = p.k_scale + kv_row;
           vs_blk = p.v_scale + kv_row;
         } else {
@@ -762,25 +794,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
 
-        // row max: four independent three-input max chains
-        float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
-        float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+        // row max: four independent three-input max chains (BS: one per 32 keys,
+        // so that the maxima of the two 64-key halves come out on the way)
+        float mx, mxh0 = 0.0f, mxh1 = 0.0f;
+        if constexpr (C::BS) {
+          float q0 = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
+          float q1 = fmaxf(__uint_as_float(sr[32]), __uint_as_float(sr[33]));
+          float q2 = fmaxf(__uint_as_float(sr[64]), __uint_as_float(sr[65]));
+          float q3 = fmaxf(__uint_as_float(sr[96]), __uint_as_float(sr[97]));
 #pragma unroll
-        for (int c = 4; c < 124; c += 8) {
-          mx0 = max3f(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-          mx1 = max3f(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-          mx2 = max3f(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-          mx3 = max3f(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+          for (int c = 2; c < 32; c += 2) {
+            q0 = max3f(q0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            q1 = max3f(q1, __uint_as_float(sr[c + 32]), __uint_as_float(sr[c + 33]));
+            q2 = max3f(q2, __uint_as_float(sr[c + 64]), __uint_as_float(sr[c + 65]));
+            q3 = max3f(q3, __uint_as_float(sr[c + 96]), __uint_as_float(sr[c + 97]));
+          }
+          mxh0 = fmaxf(q0, q1);
+          mxh1 = fmaxf(q2, q3);
+          mx = fmaxf(mxh0, mxh1);
+        } else {
+          float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+          float mx2 = __uint_as_float(sr[2]), mx3 = __uint_as_float(sr[3]);
+#pragma unroll
+          for (int c = 4; c < 124; c += 8) {
+            mx0 = max3f(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            mx1 = max3f(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+            mx2 = max3f(mx2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+            mx3 = max3f(mx3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+          }
+          mx0 = max3f(mx0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
+          mx1 = max3f(mx1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
+          mx = max3f(mx0, mx1, fmaxf(mx2, mx3));
         }
-        mx0 = max3f(mx0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
-        mx1 = max3f(mx1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
-        const float mx = max3f(mx0, mx1, fmaxf(mx2, mx3));
         float c_blk = c_log2;  // S multiplier of this block (log2 units)
         float lr = 0.0f;       // log2(sv[i] / s_ref), folded into P (per-block V scales)
         float v_alpha = 1.0f;  // O rescale when s_ref grows
         if constexpr (FP8) {
           if (p.per_block) {
-            c_blk = c_log2 * __ldg(ks_blk + i);
+            c_blk = c_log2 * (sq_blk * __ldg(ks_blk + i));  // associated as for per-head scales
             const float sv = __ldg(vs_blk + i);
             if (i == 0 || sv > v_mult) {
               if (i > 0) v_alpha = v_mult / sv;
@@ -804,6 +855,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
         // probabilities, packed in place (entry c/2 or c/4 is already consumed)
         float l_blk;
+        uint32_t sf_word = 0x7F7F7F7Fu;  // BS: UE8M0 scales of P for keys 0-31, 32-63, 64-95, 96-127
         if constexpr (!FP8) {
           const float nm = C::E_SHIFT - m_run;
           float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
@@ -835,16 +887,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           l_blk = (sa + sb) + (sc + sd);
         } else if (mma_sum) {
           // codes only; the tensor core adds them up
-          if constexpr (FMA_P) {
-            const float A = c_blk * (8.0f / 126.0f);
-            const float Bc = (8.0f * (C::E_SHIFT - m_run + lr) + 56.0f) * (1.0f / 126.0f);
+          if constexpr (C::BS) {
+            // Half h of the block is coded as 2^(x + z_h), x = c S - m_run, with the
+            // integer z_h = floor(8 - max_h x), so that its largest probability lies
+            // in (2^7, 2^8] (code <= 120). Its scale factor 2^(E - z_h) brings every
+            // half back to 2^(x + E), the common factor that O / l cancels. A half
+            // with no visible key has max_h x = -inf: z_h is clamped so the factor
+            // stays a UE8M0 number (>= 2^-127); its codes are all zero.
+            const float A = c_blk * 8.0f;
+            const float z0 = fminf(floorf(fmaf(-c_blk, mxh0, 8.0f + m_run)), 127.0f + C::E_SHIFT);
+            const float z1 = fminf(floorf(fmaf(-c_blk, mxh1, 8.0f + m_run)), 127.0f + C::E_SHIFT);
+            const float b0 = kLeanBias - 8.0f * m_run;
+            const float Bc0 = fmaf(z0, 8.0f, b0), Bc1 = fmaf(z1, 8.0f, b0);
+            const uint32_t sf0 = static_cast<uint32_t>(__float2int_rn(127.0f + C::E_SHIFT - z0));
+            const uint32_t sf1 = static_cast<uint32_t>(__float2int_rn(127.0f + C::E_SHIFT - z1));
+            sf_word = (sf0 | (sf1 << 16)) * 0x101u;
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+              const float Bc = c < 64 ? Bc0 : Bc1;
+              float w0, w1, w2, w3;
+              ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), A, Bc, w0, w1);
+              ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), A, Bc, w2, w3);
+              const uint32_t u01 = lean_codes_x2(w0, w1);
+              const uint32_t u23 = lean_codes_x2(w2, w3);
+              sr[c >> 2] = prmt(u01, u23, 0x6420u);
+            }
+          } else if constexpr (FMA_P) {
+            const float A = c_blk * 8.0f;
+            const float Bc = 8.0f * (C::E_SHIFT - m_run + lr) + kLeanBias;
 #pragma unroll
             for (int c = 0; c < 128; c += 4) {
               float w0, w1, w2, w3;
               ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), A, Bc, w0, w1);
               ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), A, Bc, w2, w3);
-              const uint32_t u01 = hfma2(pack_f16x2_relu(w0, w1), 0x57E057E0u, 0x66006600u);
-              const uint32_t u23 = hfma2(pack_f16x2_relu(w2, w3), 0x57E057E0u, 0x66006600u);
+              const uint32_t u01 = lean_codes_x2(w0, w1);
+              const uint32_t u23 = lean_codes_x2(w2, w3);
               sr[c >> 2] = prmt(u01, u23, 0x6420u);
             }
           } else {
@@ -863,17 +940,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // acc: f16x2 partial sums of decode(code)/256 (8 adds per accumulator per block)
           uint32_t acc[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
           if constexpr (FMA_P) {
-            // w = (8 (c*S - m_run + E + lr) + 56) / 126, clamped below at 0; code = round(126 w)
-            const float A = c_blk * (8.0f / 126.0f);
-            const float Bc = (8.0f * (C::E_SHIFT - m_run + lr) + 56.0f) * (1.0f / 126.0f);
+            // code = round(8 (c*S - m_run + E + lr) + 56), clamped below at 0
+            const float A = c_blk * 8.0f;
+            const float Bc = 8.0f * (C::E_SHIFT - m_run + lr) + kLeanBias;
 #pragma unroll
             for (int c = 0; c < 128; c += 4) {
               float w0, w1, w2, w3;
               ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), A, Bc, w0, w1);
               ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), A, Bc, w2, w3);
               // f16 lanes 1536 + code: bits 0x6600 + code
-              const uint32_t u01 = hfma2(pack_f16x2_relu(w0, w1), 0x57E057E0u /*126*/, 0x66006600u /*1536*/);
-              const uint32_t u23 = hfma2(pack_f16x2_relu(w2, w3), 0x57E057E0u, 0x66006600u);
+              const uint32_t u01 = lean_codes_x2(w0, w1);
+              const uint32_t u23 = lean_codes_x2(w2, w3);
               const int jj = (c >> 1) & 7;
               // (u - 0x66006600) * 128: each lane becomes code << 7
               acc[jj] = hadd2(acc[jj], u01 * 128u + 0xFFCD0000u);
@@ -938,8 +1015,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               tmem_st16(tO + DV, orr);
             }
           }
-          // P row -> its own TMEM columns
+          // P row -> its own TMEM columns (BS: and the row's scales, read by the same PV)
           tmem_st32(tP + pb * C::P_COLS, sr);
+          if constexpr (C::BS) tmem_st1(tO + C::SF_COL + (warp & 3), sf_word);
           if constexpr (!FP8) tmem_st32(tP + pb * C::P_COLS + 32, sr + 32);
         } else {
           // rescale this tile's O accumulator (PV_t,i-1 has completed: S_t,i was issued after it)

@@ -367,15 +367,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
         // e4m3 codes in place (entry c/4 is already consumed)
         if constexpr (FMA_P) {
-          const float A = c_log2 * (8.0f / 126.0f);
-          const float Bc = (8.0f * (C::E_SHIFT - m_run) + 56.0f) * (1.0f / 126.0f);
+          const float A = c_log2 * 8.0f;
+          const float Bc = 8.0f * (C::E_SHIFT - m_run) + kLeanBias;
 #pragma unroll
           for (int c = 0; c < 128; c += 4) {
             float w0, w1, w2, w3;
             ffma2_bcast(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]), A, Bc, w0, w1);
             ffma2_bcast(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]), A, Bc, w2, w3);
-            const uint32_t u01 = hfma2(pack_f16x2_relu(w0, w1), 0x57E057E0u /*126*/, 0x66006600u /*1536*/);
-            const uint32_t u23 = hfma2(pack_f16x2_relu(w2, w3), 0x57E057E0u, 0x66006600u);
+            const uint32_t u01 = lean_codes_x2(w0, w1);
+            const uint32_t u23 = lean_codes_x2(w2, w3);
             sr[c >> 2] = prmt(u01, u23, 0x6420u);
           }
         } else {

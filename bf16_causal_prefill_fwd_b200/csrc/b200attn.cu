@@ -80,11 +80,19 @@ bool make_tmap_box(CUtensorMap* m, const void* ptr, bool fp8, int d, int H, int 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // How the FP8 kernel forms e4m3 probabilities: Lean P (FMA bit construction,
-// the default) or the MUFU exponential. B200ATTN_FP8_P=mufu selects the latter;
-// read on every call so A/B runs need no rebuild.
+// the default) or the MUFU exponential; B200ATTN_FP8_P=mufu selects the latter.
+// B200ATTN_FP8_P=block selects Lean P with one power-of-two scale per 64-key
+// half block, applied by the block-scaled MMA (two-tile kernel, per-head K/V
+// scales; other configurations run Lean P). Read on every call so A/B runs
+// need no rebuild.
 bool fp8_lean_p() {
   const char* e = std::getenv("B200ATTN_FP8_P");
   return !(e && std::strcmp(e, "mufu") == 0);
+}
+
+bool fp8_block_scaled_p() {
+  const char* e = std::getenv("B200ATTN_FP8_P");
+  return e && std::strcmp(e, "block") == 0;
 }
 
 // BF16 probabilities: one exponential in four by a polynomial on the FMA pipe
@@ -122,16 +130,16 @@ bool regs_match(const void* kern) {
   return ok;
 }
 
-template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S, bool QF = false>
+template <int DQK, int DV, bool FP8, bool FMA_P, bool SHARED_S, bool QF = false, bool BSP = false>
 int launch_attn_t(const void* q, const void* k, const void* v, const AttnParams& p, int d_qk, int d_v, int sm_count,
                 cudaStream_t stream) {
-  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S, QF>;
+  using C = AttnCfg<DQK, DV, FP8, FMA_P, SHARED_S, QF, BSP>;
   CUtensorMap tq, tk, tv;
   // QF: the kernel reads Q itself (p.q_bf16); the Q map is encoded but unused.
   if (!make_tmap(&tq, q, FP8 && !QF, d_qk, p.Hq, p.N, p.B) || !make_tmap(&tk, k, FP8, d_qk, p.Hkv, p.N, p.B) ||
       !make_tmap(&tv, v, FP8, d_v, p.Hkv, p.N, p.B))
     return B200ATTN_ERR_CUDA;
-  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, FMA_P, SHARED_S, QF>;
+  auto kern = b200::attn_fwd_kernel<DQK, DV, FP8, FMA_P, SHARED_S, QF, BSP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return B200ATTN_ERR_CUDA;
   // The kernel's role split (setmaxnreg) hands out registers from the block's
@@ -359,6 +367,10 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o, int B, in
     if (d_qk == 128) return launch_attn_pair<128, 128, false>(q, k, v, p, d_qk, d_v, st);
     return launch_attn_pair<192, 128, false>(q, k, v, p, d_qk, d_v, st);
   }
+  if (!p.per_block && shared_s() && fp8_block_scaled_p()) {
+    if (d_qk == 128) return launch_attn_t<128, 128, true, true, true, false, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+    return launch_attn_t<192, 128, true, true, true, false, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+  }
   if (fp8_lean_p()) {
     if (d_qk == 128) return launch_attn<128, 128, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn<192, 128, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
@@ -482,6 +494,10 @@ int b200attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, co
     }
     if (d_qk == 128) return launch_attn<128, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn<192, 128, false>(q, k, v, p, d_qk, d_v, sm_count, st);
+  }
+  if (shared_s() && fp8_block_scaled_p()) {
+    if (d_qk == 128) return launch_attn_t<128, 128, true, true, true, false, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+    return launch_attn_t<192, 128, true, true, true, false, true>(q, k, v, p, d_qk, d_v, sm_count, st);
   }
   if (fp8_lean_p()) {
     if (d_qk == 128) return launch_attn<128, 128, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);

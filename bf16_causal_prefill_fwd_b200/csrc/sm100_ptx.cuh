@@ -233,6 +233,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// One 32-bit column per lane (32x32b.x1) and four columns of one value (x4).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void tmem_st4_same(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -350,6 +359,34 @@ __device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint
   }
 }
 
+// Block-scaled e4m3 MMA (kind::mxf8f6f4.block_scale, one UE8M0 scale per row of
+// A and per column of B for every 32 elements of K), A from tensor memory.
+// D = sum_k A[m][k] B[k][n] 2^(sfa(m) - 127) 2^(sfb(n) - 127), fp32.
+// Scale-factor operands in tensor memory, as measured on sm_100a for M = 128:
+// the scale of row m is byte sf_id of the 32-bit cell at lane m, column
+// sfa + m / 32 (columns n / 32 for B). sf_id (0..3) sits both in the
+// instruction descriptor and in bits [30,32) of the scale address, so four
+// successive K steps can read four bytes of one word.
+// Instruction descriptor: B scale id [4,6), A format [7,10) (0 = E4M3),
+// B format [10,13), B major at bit 16 (1 = MN-major), N >> 3 in [17,23),
+// scale type at bit 23 (1 = UE8M0), M >> 4 in [24,29), A scale id [29,31).
+__host__ __device__ constexpr uint32_t idesc_block_scaled(int M, int N, bool b_mn_major) {
+  return ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ts_bs_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t sf_id,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 bd, {%2, %7};\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [%1], bd, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc | (sf_id << 29)), "r"(sfa_tmem | (sf_id << 30)), "r"(sfb_tmem),
+      "r"(accumulate), "r"(kSdescHi)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ arithmetic helpers
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -451,6 +488,20 @@ __device__ __forceinline__ void fadd2(float& s0, float& s1, float a0, float a1) 
 }
 
 // Two fp32 -> f16x2 with negative values (and -inf) clamped to +0, lo in bits [0,16).
+// Lean P codes of two probabilities. v = 8 x + 56 + 1536 for p = 2^x: the
+// convert to f16x2 rounds v to the nearest integer in one step (f16 spacing is 1
+// in [1024, 2048)), so each 16-bit lane reads 0x6600 + round(8 x + 56) once the
+// f16x2 max against 1536 has clamped codes below zero to 0. The low byte of each
+// lane is the e4m3 code; lo in bits [0,16).
+constexpr float kLeanBias = 56.0f + 1536.0f;
+
+__device__ __forceinline__ uint32_t lean_codes_x2(float v_lo, float v_hi) {
+  uint32_t h, r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(v_hi), "f"(v_lo));
+  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x66006600u));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2_relu(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.relu.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -53,9 +53,11 @@ SMALL = [
 ]
 
 
-# The FP8 kernel forms e4m3 probabilities either with the MUFU exponential or
-# with Lean P (FMA bit construction); both are tested.
-FP8_P = ["lean", "mufu"]
+# The FP8 kernel forms e4m3 probabilities with the MUFU exponential, with Lean P
+# (FMA bit construction), or with Lean P and one power-of-two scale per 64-key
+# half block applied by the block-scaled MMA ("block": the two-tile kernel with
+# per-head K/V scales; elsewhere it runs Lean P); all three are tested.
+FP8_P = ["lean", "mufu", "block"]
 
 
 # FP8 with per-head scales has three kernels: both query tiles of a unit on one
@@ -122,6 +124,10 @@ MUFU_LSE_ATOL = 0.061
 LEAN_LSE_ATOL = 0.121
 
 
+def lse_atol(fp8_p):
+    return MUFU_LSE_ATOL if fp8_p == "mufu" else LEAN_LSE_ATOL
+
+
 @pytest.mark.parametrize("bf16_p", BF16_P, indirect=True)
 @pytest.mark.parametrize("shape", SMALL)
 @pytest.mark.parametrize("causal", [True, False])
@@ -141,6 +147,8 @@ def test_bf16_matches_oracle(shape, causal, bf16_p):
 @pytest.mark.parametrize("shape", SMALL)
 @pytest.mark.parametrize("causal", [True, False])
 def test_fp8_matches_oracle(shape, causal, fp8_p, fp8_kernel):
+    if fp8_p == "block" and fp8_kernel != "two":
+        pytest.skip("block-scaled P is built into the two-tile kernel only")
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq + 1))
     codes, deq = oracle_fp8_inputs(q, k, v)
@@ -148,7 +156,7 @@ def test_fp8_matches_oracle(shape, causal, fp8_p, fp8_kernel):
     ref, ref_lse = oracle.attention(*deq, causal=causal)
     err = oracle.rel_rms(f32(o), ref)
     assert err <= FP8_TOL, err
-    check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
+    check_lse(lse, ref_lse, atol=lse_atol(fp8_p))
 
 
 PER_BLOCK_SHAPES = [(1, 4, 2, 300, 128), (2, 2, 1, 700, 128), (1, 4, 4, 520, 192)]
@@ -173,7 +181,7 @@ def test_fp8_per_block_scales_match_oracle(shape, causal, fp8_p):
     ref, ref_lse = oracle.attention(*deq, causal=causal)
     err = oracle.rel_rms(f32(o), ref)
     assert err <= FP8_TOL, err
-    check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
+    check_lse(lse, ref_lse, atol=lse_atol(fp8_p))
 
 
 Q_BLOCK_SHAPES = [(1, 4, 2, 300, 128), (2, 8, 2, 1000, 128), (1, 4, 4, 520, 192)]
@@ -200,7 +208,7 @@ def test_fp8_q_block_scales_match_oracle(shape, causal, fp8_p):
     ref, ref_lse = oracle.attention(*deq, causal=causal)
     err = oracle.rel_rms(f32(o), ref)
     assert err <= FP8_TOL, err
-    check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL if fp8_p == "lean" else MUFU_LSE_ATOL)
+    check_lse(lse, ref_lse, atol=lse_atol(fp8_p))
 
 
 def test_full_size_fp8_q_block_sampled():
@@ -269,6 +277,37 @@ def test_tiny_workload_both_dtypes(fp8_p):
     assert e_bf16 <= BF16_TOL and e_fp8 <= FP8_TOL
 
 
+@pytest.mark.parametrize("dqk", [128, 192])
+def test_fp8_block_scaled_p_keeps_small_halves(dqk, monkeypatch):
+    """One dominant key per row and 255 keys 2^-12 below it. Lean P codes every
+    probability as 2^(x - m + 4) against the row's running max m, so the small
+    ones land at 2^-8, below the smallest code its formula reaches (2^-7), and
+    are dropped. Block-scaled P puts the largest probability of each 64-key half
+    at 2^8: the dominant key's half keeps its small keys at 2^-4, and the three
+    other halves code theirs exactly. Only those three halves carry V = 1, so the
+    output is 192 / (2^12 + 255) per element, which Lean P returns as 0."""
+    N = 256
+    q = torch.zeros(1, N, 1, dqk)
+    q[..., 0] = 1.0
+    k = torch.zeros(1, N, 1, dqk)
+    k[:, 0, :, 0] = 4.0
+    v = torch.zeros(1, N, 1, 128)
+    v[:, 64:] = 1.0
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    codes, deq = oracle_fp8_inputs(q, k, v)
+    scale = 3.0 * np.log(2.0)  # score gap 4 * scale = 12 in log2 units
+    ref, ref_lse = oracle.attention(*deq, causal=False, softmax_scale=scale)
+    errs = {}
+    for mode in ("lean", "block"):
+        monkeypatch.setenv("B200ATTN_FP8_P", mode)
+        o, lse = run_fp8(codes, causal=False, scale=scale)
+        errs[mode] = oracle.rel_rms(f32(o), ref)
+    print(f"one dominant key, d_qk={dqk}: rel RMS lean {errs['lean']:.3e}, block {errs['block']:.3e}")
+    assert errs["lean"] > 0.9       # the small probabilities are all lost
+    assert errs["block"] < 0.01     # every code is exact here; what is left is the bf16 output
+    check_lse(lse, ref_lse, atol=LEAN_LSE_ATOL)
+
+
 def test_explicit_softmax_scale():
     q, k, v = workloads.draw(workloads.gaussian(1, 2, 1, 200, 128, 128, seed=5))
     o, lse = run_bf16(q, k, v, scale=0.02)
@@ -322,6 +361,8 @@ def test_bf16_many_units_per_cta(causal, bf16_p):
 @pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
 @pytest.mark.parametrize("causal", [True, False])
 def test_fp8_many_units_per_cta(causal, fp8_p, fp8_kernel):
+    if fp8_p == "block" and fp8_kernel != "two":
+        pytest.skip("block-scaled P is built into the two-tile kernel only")
     B, Hq, Hkv, N, dqk = MANY_UNITS
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=22))
     codes, deq = oracle_fp8_inputs(q, k, v)
@@ -333,7 +374,8 @@ def test_fp8_many_units_per_cta(causal, fp8_p, fp8_kernel):
     assert err <= FP8_TOL, err
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "bf16-mixed", "fp8-lean", "fp8-mufu", "fp8-lean-pair", "fp8-lean-tile"])
+@pytest.mark.parametrize("dtype", ["bf16", "bf16-mixed", "fp8-lean", "fp8-mufu", "fp8-block", "fp8-lean-pair",
+                                   "fp8-lean-tile"])
 def test_bitwise_deterministic_over_1000_launches(dtype, monkeypatch):
     monkeypatch.setenv("B200ATTN_BF16_P", "mixed" if dtype == "bf16-mixed" else "mufu")
     if dtype.startswith("fp8"):
@@ -416,7 +458,7 @@ def test_full_size_fp8_sampled(name, hadamard, monkeypatch):
 
 
 @pytest.mark.parametrize("fp8_kernel", ["pair", "tile"], indirect=True)
-@pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
+@pytest.mark.parametrize("fp8_p", ["lean", "mufu"], indirect=True)
 def test_full_size_fp8_other_kernels_sampled(fp8_p, fp8_kernel):
     """The FP8 kernels other than the default on the full 7B-style layer
     (N = 16384), where their K/V rings wrap many times per unit."""
