@@ -61,8 +61,8 @@ def parse_args():
                          "quantizer per head (separate), or by the quantizer per 128-token block in one pass "
                          "(qblock); K and V per head by the quantizer")
     ap.add_argument("--fp8-p", choices=["lean", "mufu", "block"], default=None,
-                    help="how the FP8 kernel forms probabilities (default: the library default, Lean P; block = "
-                         "Lean P with one power-of-two scale per 64-key half block, applied by the block-scaled MMA)")
+                    help="how the FP8 kernel forms probabilities (default: the library default, block = Lean P "
+                         "with one power-of-two scale per 64-key half block, applied by the block-scaled MMA)")
     ap.add_argument("--settle-s", type=float, default=1.0,
                     help="untimed back-to-back steps before timing so clocks reach their sustained level")
     ap.add_argument("--no-e2e", action="store_true")
@@ -338,6 +338,16 @@ def fp8_step_desc(args) -> str:
     return "e4m3 quantizer on Q,K,V (" + q + (", Hadamard on Q,K" if had else "") + ") + FP8 attention"
 
 
+def fp8_p_desc(args) -> str:
+    """How the FP8 attention kernel of the step forms its probabilities."""
+    env_p = os.environ.get("B200ATTN_FP8_P")
+    if env_p == "mufu":
+        return "mufu"
+    if env_p == "lean" or args.fp8_q == "fused" or os.environ.get("B200ATTN_SHARED_S") == "0":
+        return "lean"
+    return "lean, block-scaled (power-of-two scale per 64-key half block)"
+
+
 def run_config(args, w: workloads.Workload, world: int) -> dict:
     """The `config` object of the JSON line; both arms print the same one."""
     return {"workload": workload_desc(w),
@@ -345,7 +355,7 @@ def run_config(args, w: workloads.Workload, world: int) -> dict:
             "flops_per_step": w.flops, "flop_convention": "B*Hq*N^2*(d_qk+d_v)",
             "l2": "256 MiB buffer written between timed steps (untimed); inputs exceed L2",
             "settle": f"{args.settle_s} s of untimed back-to-back steps before timing",
-            "fp8_p": (os.environ.get("B200ATTN_FP8_P") or "lean") if args.dtype == "fp8" else None,
+            "fp8_p": fp8_p_desc(args) if args.dtype == "fp8" else None,
             "parallelism": f"replicas x{world}"}
 
 
@@ -505,7 +515,7 @@ def kernel_name(dtype: str, w: workloads.Workload, fused_q: bool = False) -> str
             kname = "attn_fwd_pair_kernel"
         else:
             kname = "attn_fwd_kernel"
-            if env_p == "block" and os.environ.get("B200ATTN_SHARED_S") != "0":
+            if env_p not in ("lean", "mufu") and os.environ.get("B200ATTN_SHARED_S") != "0":
                 fp8_p = "lean,block-scaled"
         return f"{kname}<{w.d_qk},{w.d_v},fp8,{fp8_p}>"
     bf16_p = "mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed"

@@ -204,6 +204,11 @@ struct AttnCfg {
       BS ? idesc_block_scaled(kBM, DVX, true) : idesc_dense(FP8 ? 0u : 1u, FP8 ? 0u : 1u, kBM, DVX, true);
   static_assert(!BSP || (FP8 && FMA_P && RS), "block-scaled P is a variant of Lean P with tensor-core row sums");
   static_assert(!BS || SFB_COLS >= 8, "B scales need the columns n / 32 of N = d_v + 16");
+  // Register split. The block-scaled PV issue with d_qk = 192 needs a few more
+  // registers in the issuer warps than 72 (it spilled there); its softmax fits in 200.
+  static constexpr int REGS_LOW = BS && DQK > 128 ? 80 : kRegsLow;
+  static constexpr int REGS_HIGH = BS && DQK > 128 ? 200 : kRegsHigh;
+  static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= kAttnThreads * kRegsAtLaunch, "register split");
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
   static_assert(SK >= 2 && SV >= 1, "K/V rings");
   static_assert(!SS || TM_P + 2 * PB * P_COLS <= 512, "TMEM budget");
@@ -418,8 +423,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // Register split between roles: the producer and issuer warps need few
     // registers, the softmax warps hold a 128-entry score row each. The block
     // is launched with kRegsAtLaunch per thread (the host checks), and
-    // 128 * kRegsLow + 256 * kRegsHigh does not exceed 384 * kRegsAtLaunch.
-    setmaxnreg_dec<kRegsLow>();
+    // 128 * REGS_LOW + 256 * REGS_HIGH does not exceed 384 * kRegsAtLaunch.
+    setmaxnreg_dec<C::REGS_LOW>();
   if (warp == 0 || warp == 3) {
     // ------------------------------------------------------------ TMA producers
     // warp 0: Q tiles and K blocks; warp 3: V blocks. Each walks the same unit
@@ -647,7 +652,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   }
   } else {
-    setmaxnreg_inc<kRegsHigh>();
+    setmaxnreg_inc<C::REGS_HIGH>();
     // ------------------------------------------------------------ softmax + epilogue
     const int t = (warp - 4) >> 2;            // query tile of this warpgroup
     const int r = threadIdx.x - 128 - 128 * t;  // row within the tile == TMEM lane

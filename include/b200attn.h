@@ -73,6 +73,13 @@ enum {
  * BF16, head dim 128 and 192/128, flash_attn_func drop-in) and "ZYFA 如何工作？"
  * (FP8 probabilities, divide by the row sum of the probabilities actually used).
  *
+ * FP8 probabilities are e4m3 codes formed without an exponential (Lean P). With
+ * per-head K/V scales (SCALE_PER_HEAD, SCALE_Q_BLOCK) each 64-key half of a key
+ * block carries its own power-of-two scale, applied by the block-scaled tensor-
+ * core MMA ("逐块缩放与舍入行和"); with SCALE_PER_BLOCK each row carries one
+ * exponent shift. The environment variable B200ATTN_FP8_P, read on every call,
+ * selects one shift per row (=lean) or the exponential rounded to e4m3 (=mufu).
+ *
  * q      [B, N, Hq,  d_qk]  bf16, or e4m3 codes when dtype == FP8_E4M3
  * k      [B, N, Hkv, d_qk]  same dtype as q
  * v      [B, N, Hkv, d_v]   same dtype as q
