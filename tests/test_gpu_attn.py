@@ -245,9 +245,12 @@ def test_full_size_fp8_q_block_sampled():
 ROW_SUM_UNIT_TOL = 8 * 2.0 ** -11
 
 
-def test_fp8_per_block_matches_per_head_when_scales_agree():
+def test_fp8_per_block_matches_per_head_when_scales_agree(monkeypatch):
     """Per-block scales that all equal the per-head scale give the per-head output
-    up to the rounding of the row sum."""
+    up to the rounding of the row sum. Both calls form probabilities with one
+    exponent shift per row (Lean P), so that the codes are the same; per-head
+    scales would otherwise take the block-scaled probabilities."""
+    monkeypatch.setenv("B200ATTN_FP8_P", "lean")
     q, k, v = workloads.draw(workloads.gaussian(1, 4, 2, 384, 128, 128, seed=9))
     codes, _ = oracle_fp8_inputs(q, k, v, granularity="head")
     q8, sq, k8, sk, v8, sv = to_gpu_fp8(codes)
