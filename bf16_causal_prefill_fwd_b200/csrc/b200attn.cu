@@ -283,6 +283,13 @@ int launch_quant_qkv(const b200::QkvQuant& a, int B, int gran, cudaStream_t stre
     } else if (DQK == 128 && DV == 128) {
       b200::quant_qkv_absmax_group_kernel<HAD, 1><<<grid, b200::kQuantThreads, 0, stream>>>(a);
       b200::quant_qkv_encode_group_kernel<HAD, 1><<<grid, b200::kQuantThreads, 0, stream>>>(a);
+    } else if (DQK == 192 && DV == 128 && a.H[0] % 2 == 0 && a.H[1] % 2 == 0 && a.H[2] % 2 == 0) {
+      const dim3 ggrid(grid.x / 2, a.nblk, B);
+      b200::quant_qkv_absmax_group_mla_kernel<HAD, 2><<<ggrid, b200::kQuantThreads, 0, stream>>>(a);
+      b200::quant_qkv_encode_group_mla_kernel<HAD, 2><<<ggrid, b200::kQuantThreads, 0, stream>>>(a);
+    } else if (DQK == 192 && DV == 128) {
+      b200::quant_qkv_absmax_group_mla_kernel<HAD, 1><<<grid, b200::kQuantThreads, 0, stream>>>(a);
+      b200::quant_qkv_encode_group_mla_kernel<HAD, 1><<<grid, b200::kQuantThreads, 0, stream>>>(a);
     } else {
       b200::quant_qkv_absmax_kernel<DQK, DV, HAD><<<grid, b200::kQuantThreads, 0, stream>>>(a);
       b200::quant_qkv_encode_kernel<DQK, DV, HAD, true><<<grid, b200::kQuantThreads, 0, stream>>>(a);

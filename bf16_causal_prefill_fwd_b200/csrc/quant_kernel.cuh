@@ -165,12 +165,71 @@ __device__ __forceinline__ void absmax_body(const __nv_bfloat16* __restrict__ x,
   if (threadIdx.x == 0) partial[(static_cast<size_t>(b) * H + h) * nblk + blk] = m;
 }
 
+// One-pass encode of one 128-token block with its own scale, no rotation: no
+// lane layout is needed, so the block is read as 16-byte chunks, consecutive
+// chunks on consecutive threads and every lane loading (the d = 192 row layout
+// of the rotation leaves half the lanes of each load idle). Codes and scale are
+// those of encode_body<D, false, false>, bit for bit.
+template <int D>
+__device__ __forceinline__ void encode_block_flat_body(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
+                                                       float* __restrict__ scale, int N, int H, int nblk, int blk,
+                                                       int h, int b, float* red) {
+  constexpr int kChunksPerRow = D / 8;  // 16-byte chunks (8 bf16) in a row
+  constexpr int kPer = kQuantBlock * kChunksPerRow / kQuantThreads;
+  static_assert(kQuantBlock * kChunksPerRow % kQuantThreads == 0, "whole chunks per thread");
+  const int tid = threadIdx.x;
+  uint4 raw[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int c = tid + i * kQuantThreads;
+    const int row = blk * kQuantBlock + c / kChunksPerRow, rc = row < N ? row : N - 1;
+    raw[i] = *reinterpret_cast<const uint4*>(x + ((static_cast<size_t>(b) * N + rc) * H + h) * D +
+                                             8 * (c % kChunksPerRow));
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i)
+    asm volatile("" : "+r"(raw[i].x), "+r"(raw[i].y), "+r"(raw[i].z), "+r"(raw[i].w));
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int row = blk * kQuantBlock + (tid + i * kQuantThreads) / kChunksPerRow;
+    if (row < N) {
+      float v[8];
+      bf16x8_to_float(raw[i], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+    }
+  }
+  const float amax = block_max(m, red);
+  const bool pos = amax > 0.0f;
+  const float inv = pos ? __fdiv_rn(448.0f, amax) : 1.0f;
+  if (tid == 0) scale[(static_cast<size_t>(b) * H + h) * nblk + blk] = pos ? __fdiv_rn(amax, 448.0f) : 1.0f;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int c = tid + i * kQuantThreads;
+    const int row = blk * kQuantBlock + c / kChunksPerRow;
+    if (row < N) {
+      float v[8];
+      bf16x8_to_float(raw[i], v);
+      uint32_t q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q[j] = pack_e4m3x2(__fmul_rn(v[2 * j], inv), __fmul_rn(v[2 * j + 1], inv));
+      *reinterpret_cast<uint2*>(y + ((static_cast<size_t>(b) * N + row) * H + h) * D + 8 * (c % kChunksPerRow)) =
+          make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+    }
+  }
+}
+
 // Encode one 128-token block. PER_HEAD: amax is the max of the partials of
 // this head; otherwise the block's own.
 template <int D, bool HAD, bool PER_HEAD>
 __device__ __forceinline__ void encode_body(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y,
                                             float* __restrict__ scale, const float* __restrict__ partial, int N,
                                             int H, int nblk, int blk, int h, int b, float* red) {
+  if constexpr (D == 192 && !HAD && !PER_HEAD) {
+    encode_block_flat_body<D>(x, y, scale, N, H, nblk, blk, h, b, red);
+    return;
+  }
   using L = QuantLayout<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint4 raw[L::ITERS];
@@ -280,25 +339,30 @@ __device__ __forceinline__ T pick3(const T (&arr)[3], int t) {  // no dynamic in
   return t == 0 ? arr[0] : (t == 1 ? arr[1] : arr[2]);
 }
 
+// Which tensor (0 Q, 1 K, 2 V) and which group of G heads of it CTA x covers.
+template <int G>
+__device__ __forceinline__ int qkv_group(const QkvQuant& a, int x, int& g) {
+  const int gq = a.H[0] / G, gk = a.H[1] / G;
+  if (x < gq) {
+    g = x;
+    return 0;
+  }
+  if (x < gq + gk) {
+    g = x - gq;
+    return 1;
+  }
+  g = x - gq - gk;
+  return 2;
+}
+
+// red: kQuantThreads / 32 * 4 floats of shared memory.
 template <bool HAD, int G>
-__global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_kernel(const QkvQuant a) {
+__device__ __forceinline__ void absmax_group_body(const QkvQuant& a, int t, int g, float* red) {
   constexpr int kChunks = 16 * G;             // 16-byte segments in a row of the group
   constexpr int kRowsPerStep = kQuantThreads / kChunks;
   constexpr int kSteps = kQuantBlock / kRowsPerStep;
   static_assert(kSteps % 8 == 0, "steps are loaded eight at a time");
-  __shared__ float red[kQuantThreads / 32][2];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = a.H[0] / G, gk = a.H[1] / G;
-  int t, g = blockIdx.x;
-  if (g < gq) {
-    t = 0;
-  } else if (g < gq + gk) {
-    t = 1;
-    g -= gq;
-  } else {
-    t = 2;
-    g -= gq + gk;
-  }
   const int H = pick3(a.H, t), N = a.N, blk = blockIdx.y, b = blockIdx.z;
   const int r_in = tid / kChunks;
   const uint4* base = reinterpret_cast<const uint4*>(pick3(a.x, t)) + static_cast<size_t>(b) * N * H * 16 +
@@ -325,7 +389,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_kernel(c
   }
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));  // within a half-warp
-  if ((lane & 15) == 0) red[warp][lane >> 4] = m;
+  if ((lane & 15) == 0) red[2 * warp + (lane >> 4)] = m;
   __syncthreads();
   if (tid < G) {  // head tid of the group
     float mh = 0.0f;
@@ -333,9 +397,17 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_kernel(c
     for (int w = 0; w < kQuantThreads / 32; ++w)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
-        if (((w * 32 + hh * 16) % kChunks) / 16 == tid) mh = fmaxf(mh, red[w][hh]);
+        if (((w * 32 + hh * 16) % kChunks) / 16 == tid) mh = fmaxf(mh, red[2 * w + hh]);
     pick3(a.partial, t)[(static_cast<size_t>(b) * H + g * G + tid) * a.nblk + blk] = mh;
   }
+}
+
+template <bool HAD, int G>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_kernel(const QkvQuant a) {
+  __shared__ float red[kQuantThreads / 32 * 4];
+  int g;
+  const int t = qkv_group<G>(a, blockIdx.x, g);
+  absmax_group_body<HAD, G>(a, t, g, red);
 }
 
 // Pass 2 (per-head scales) over Q, K and V for d_qk = d_v = 128, on the grid and
@@ -345,24 +417,13 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_kernel(c
 // time. The first loads are issued before the partial maxima are reduced.
 // Codes and scales are those of quant_qkv_encode_kernel, bit for bit.
 template <bool HAD, int G>
-__global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_group_kernel(const QkvQuant a) {
+__device__ __forceinline__ void encode_group_body(const QkvQuant& a, int t, int g, float* red) {
   constexpr int kChunks = 16 * G;
   constexpr int kRowsPerStep = kQuantThreads / kChunks;
   constexpr int kSteps = kQuantBlock / kRowsPerStep;
   static_assert(kSteps % 8 == 0, "steps are loaded eight at a time");
-  __shared__ float red[kQuantThreads / 32][G];
+  static_assert(G <= 4, "red holds 4 values per warp");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = a.H[0] / G, gk = a.H[1] / G;
-  int t, g = blockIdx.x;
-  if (g < gq) {
-    t = 0;
-  } else if (g < gq + gk) {
-    t = 1;
-    g -= gq;
-  } else {
-    t = 2;
-    g -= gq + gk;
-  }
   const int H = pick3(a.H, t), N = a.N, blk = blockIdx.y, b = blockIdx.z;
   const int r_in = tid / kChunks, hl = (tid % kChunks) / 16;
   const size_t first = static_cast<size_t>(b) * N * H * 16 + static_cast<size_t>(g) * kChunks + tid % kChunks;
@@ -385,14 +446,14 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_group_kernel(c
     for (int i = tid; i < a.nblk; i += kQuantThreads) mh[j] = fmaxf(mh[j], ph[static_cast<size_t>(j) * a.nblk + i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mh[j] = fmaxf(mh[j], __shfl_xor_sync(0xffffffffu, mh[j], o));
-    if (lane == 0) red[warp][j] = mh[j];
+    if (lane == 0) red[4 * warp + j] = mh[j];
   }
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < G; ++j) {
-    mh[j] = red[0][j];
+    mh[j] = red[j];
 #pragma unroll
-    for (int w = 1; w < kQuantThreads / 32; ++w) mh[j] = fmaxf(mh[j], red[w][j]);
+    for (int w = 1; w < kQuantThreads / 32; ++w) mh[j] = fmaxf(mh[j], red[4 * w + j]);
   }
   float amax = mh[0];
 #pragma unroll
@@ -429,6 +490,171 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_group_kernel(c
       }
     }
   }
+}
+
+template <bool HAD, int G>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_group_kernel(const QkvQuant a) {
+  __shared__ float red[kQuantThreads / 32 * 4];
+  int g;
+  const int t = qkv_group<G>(a, blockIdx.x, g);
+  encode_group_body<HAD, G>(a, t, g, red);
+}
+
+// The per-head passes for d = 192 rows (Q and K at the MLA shape), on the
+// streaming plan of the d = 128 group kernels: a CTA takes a group of G
+// consecutive heads and one 128-token block, each warp holds one head row per
+// step in the lane layout of the rotation (lanes 0-15: 8 of the first 128
+// elements, lanes 16-31: 4 of the 64-wide tail), warp w sees head w % G of
+// the group, and eight steps of loads are in flight. Maxima, codes and scales
+// are those of absmax_body / encode_body for d = 192, bit for bit.
+template <int G>
+struct Group192 {
+  static_assert(8 % G == 0, "a step is 8 warps");
+  static constexpr int kRowsPerStep = kQuantThreads / 32 / G;
+  static constexpr int kSteps = kQuantBlock / kRowsPerStep;
+  static_assert(kSteps % 8 == 0, "steps are loaded eight at a time");
+};
+
+template <bool HAD, int G>
+__device__ __forceinline__ void absmax_group192_body(const QkvQuant& a, int t, int g, float* red) {
+  using L = Group192<G>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = pick3(a.H, t), N = a.N, blk = blockIdx.y, b = blockIdx.z;
+  const int r_in = warp / G;
+  const __nv_bfloat16* base =
+      pick3(a.x, t) + static_cast<size_t>(b) * N * H * 192 + static_cast<size_t>(g * G + warp % G) * 192;
+  float m = 0.0f;
+#pragma unroll 1
+  for (int s0 = 0; s0 < L::kSteps; s0 += 8) {
+    uint4 r[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int row = blk * kQuantBlock + (s0 + k) * L::kRowsPerStep + r_in;
+      r[k] = load_lane_raw<192>(base + static_cast<size_t>(row < N ? row : N - 1) * H * 192, lane);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float v[8];
+      lane_values<192, HAD>(r[k], lane, v);
+      if (blk * kQuantBlock + (s0 + k) * L::kRowsPerStep + r_in < N) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (tid < G) {  // head tid of the group: warps tid, tid + G, ...
+    float mh = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kQuantThreads / 32; ++w)
+      if (w % G == tid) mh = fmaxf(mh, red[w]);
+    pick3(a.partial, t)[(static_cast<size_t>(b) * H + g * G + tid) * a.nblk + blk] = mh;
+  }
+}
+
+template <bool HAD, int G>
+__device__ __forceinline__ void encode_group192_body(const QkvQuant& a, int t, int g, float* red) {
+  using L = Group192<G>;
+  static_assert(G <= 4, "red holds 4 values per warp");
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = pick3(a.H, t), N = a.N, blk = blockIdx.y, b = blockIdx.z;
+  const int r_in = warp / G, hl = warp % G;
+  const size_t first = static_cast<size_t>(b) * N * H * 192 + static_cast<size_t>(g * G + hl) * 192;
+  const __nv_bfloat16* src = pick3(a.x, t) + first;
+  uint8_t* dst = pick3(a.y, t) + first;
+
+  uint4 r[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int row = blk * kQuantBlock + k * L::kRowsPerStep + r_in;
+    r[k] = load_lane_raw<192>(src + static_cast<size_t>(row < N ? row : N - 1) * H * 192, lane);
+  }
+
+  // amax of each head of the group: the max of its partials
+  const float* ph = pick3(a.partial, t) + (static_cast<size_t>(b) * H + g * G) * a.nblk;
+  float mh[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    mh[j] = 0.0f;
+    for (int i = tid; i < a.nblk; i += kQuantThreads) mh[j] = fmaxf(mh[j], ph[static_cast<size_t>(j) * a.nblk + i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mh[j] = fmaxf(mh[j], __shfl_xor_sync(0xffffffffu, mh[j], o));
+    if (lane == 0) red[4 * warp + j] = mh[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    mh[j] = red[j];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) mh[j] = fmaxf(mh[j], red[4 * w + j]);
+  }
+  float amax = mh[0];
+#pragma unroll
+  for (int j = 1; j < G; ++j) amax = hl == j ? mh[j] : amax;
+  const float inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  if (blk == 0 && tid < G) {
+    float as = mh[0];
+#pragma unroll
+    for (int j = 1; j < G; ++j) as = tid == j ? mh[j] : as;
+    pick3(a.scale, t)[static_cast<size_t>(b) * H + g * G + tid] = as > 0.0f ? __fdiv_rn(as, 448.0f) : 1.0f;
+  }
+
+#pragma unroll 1
+  for (int s0 = 0; s0 < L::kSteps; s0 += 8) {
+    if (s0 > 0) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int row = blk * kQuantBlock + (s0 + k) * L::kRowsPerStep + r_in;
+        r[k] = load_lane_raw<192>(src + static_cast<size_t>(row < N ? row : N - 1) * H * 192, lane);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float v[8];
+      lane_values<192, HAD>(r[k], lane, v);
+      const int row = blk * kQuantBlock + (s0 + k) * L::kRowsPerStep + r_in;
+      if (row < N) {
+        uint32_t c[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          c[q] = pack_e4m3x2(__fmul_rn(v[2 * q], inv), __fmul_rn(v[2 * q + 1], inv));
+        uint8_t* d = dst + static_cast<size_t>(row) * H * 192;
+        if (lane < 16) {
+          *reinterpret_cast<uint2*>(d + 8 * lane) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+        } else {
+          *reinterpret_cast<uint32_t*>(d + 128 + 4 * (lane - 16)) = c[0] | (c[1] << 16);
+        }
+      }
+    }
+  }
+}
+
+// The per-head passes at the MLA shape (d_qk = 192, d_v = 128) in one launch
+// each: CTAs over the head groups of Q and K take the d = 192 bodies, those
+// over V's the d = 128 ones. Rotation (HAD) on Q and K only.
+template <bool HAD, int G>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_absmax_group_mla_kernel(const QkvQuant a) {
+  __shared__ float red[kQuantThreads / 32 * 4];
+  int g;
+  const int t = qkv_group<G>(a, blockIdx.x, g);
+  if (t == 2)
+    absmax_group_body<false, G>(a, 2, g, red);
+  else
+    absmax_group192_body<HAD, G>(a, t, g, red);
+}
+
+template <bool HAD, int G>
+__global__ void __launch_bounds__(kQuantThreads) quant_qkv_encode_group_mla_kernel(const QkvQuant a) {
+  __shared__ float red[kQuantThreads / 32 * 4];
+  int g;
+  const int t = qkv_group<G>(a, blockIdx.x, g);
+  if (t == 2)
+    encode_group_body<false, G>(a, 2, g, red);
+  else
+    encode_group192_body<HAD, G>(a, t, g, red);
 }
 
 template <int DQK, int DV, bool HAD, bool PER_HEAD>

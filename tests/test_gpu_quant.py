@@ -63,9 +63,11 @@ def test_full_size_single_tensor_bit_exact(name, hadamard):
 
 
 # (2, 4000, 8, 2, 128) has more 128-token head blocks (768) than the persistent
-# per-head amax pass has CTAs, so each CTA loops over several.
+# per-head amax pass has CTAs, so each CTA loops over several. The d_qk = 192
+# shapes take the MLA-shape passes: two heads per CTA when every head count is
+# even, one otherwise (3 and 1 heads).
 @pytest.mark.parametrize("shape", [(1, 300, 4, 2, 128), (2, 129, 2, 2, 192), (1, 1000, 8, 1, 128),
-                                   (2, 4000, 8, 2, 128)])
+                                   (2, 4000, 8, 2, 128), (1, 300, 3, 1, 192), (1, 1000, 8, 4, 192)])
 @pytest.mark.parametrize("granularity", ["head", "block", "q_block"])
 @pytest.mark.parametrize("hadamard", [False, True])
 def test_qkv_in_one_launch_bit_exact(shape, granularity, hadamard):
@@ -101,7 +103,7 @@ def test_kv_only_quantizer_bit_exact(hadamard):
         assert np.array_equal(c.view(torch.uint8).cpu().numpy(), ref_codes)
 
 
-@pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("qknorm", True)])
+@pytest.mark.parametrize("name,hadamard", [("gqa7b", False), ("qknorm", True), ("mla", False), ("mla", True)])
 def test_full_size_qkv_bit_exact(name, hadamard):
     """The merged quantizer at full size, in the launch configuration of the FP8
     step: K and V equal the oracle's codes and scales; Q equals the per-tensor
