@@ -515,7 +515,9 @@ def kernel_name(dtype: str, w: workloads.Workload, fused_q: bool = False) -> str
             kname = "attn_fwd_pair_kernel"
         else:
             kname = "attn_fwd_kernel"
-            if env_p not in ("lean", "mufu") and os.environ.get("B200ATTN_SHARED_S") != "0":
+            if os.environ.get("B200ATTN_SHARED_S") == "0":
+                fp8_p += ",private-S"
+            elif env_p not in ("lean", "mufu"):
                 fp8_p = "lean,block-scaled"
         return f"{kname}<{w.d_qk},{w.d_v},fp8,{fp8_p}>"
     bf16_p = "mufu" if os.environ.get("B200ATTN_BF16_P") == "mufu" else "mixed"

@@ -163,9 +163,16 @@ struct AttnCfg {
   // of ones, so columns d_v.. of O_t accumulate sum_j P_ij with the same
   // rescales as O.
   static constexpr bool RS = SS && FP8;
+  // SP (FP8 without the shared S buffer): one S buffer per tile in TMEM, so a
+  // tile's next QK^T waits only for its own S copy-out; P goes to shared memory
+  // (two buffers per tile, K-major, 128-byte swizzle) and PV reads it there (SS
+  // MMA); the row sums are kept in registers. TMEM: S_0, S_1, O_0, O_1 (512).
+  static constexpr bool SP = !SS && FP8;
   static constexpr int DVX = DV + (RS ? 16 : 0);     // O_t columns (output, then row sum)
-  static constexpr int PB = SS ? (FP8 && !RS ? 2 : 1) : 0;  // P buffers per tile
-  static constexpr int PBX = SS ? PB : 1;            // P-full / P-done barriers per tile
+  static constexpr int PB = SS ? (FP8 && !RS ? 2 : 1) : (SP ? 2 : 0);  // P buffers per tile
+  static constexpr int PBX = SS || SP ? PB : 1;      // P-full / P-done barriers per tile
+  static constexpr int P_BYTES = kBM * kBN * ESZ;    // SP: one P tile in shared memory
+  static constexpr int P_SMEM = SP ? 2 * PB * P_BYTES : 0;
   static constexpr int O_STRIDE = (DVX + 31) / 32 * 32;  // TMEM columns per O_t, kept 32-aligned
   static constexpr int TM_O = SS ? 128 : 256;        // O_t at TM_O + O_STRIDE t
   static constexpr int TM_P = SS ? 128 + 2 * O_STRIDE : 384;  // SS: P(t, b) at TM_P + P_COLS (PB t + b)
@@ -177,13 +184,13 @@ struct AttnCfg {
   // writing it between units (the encode then sits in the middle of the
   // softmax's pipeline and the K ring loses a stage), so one is used.
   static constexpr int Q_BUFS = 1;
-  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BUFS * Q_BYTES - ONES_BYTES;
+  static constexpr int RING_AVAIL = SMEM_AVAIL - 2 * Q_BUFS * Q_BYTES - ONES_BYTES - P_SMEM;
   static constexpr int RING_PAIRS = RING_AVAIL / (K_BYTES + V_BYTES);
   static constexpr int SV = RING_PAIRS >= 2 ? (RING_PAIRS > 4 ? 4 : RING_PAIRS) : 1;
   static constexpr int SK_FIT = (RING_AVAIL - SV * V_BYTES) / K_BYTES;
   static constexpr int SK = SK_FIT > 6 ? 6 : SK_FIT;
   static constexpr int NUM_BARS = 4 + 4 + 2 * SK + 2 * SV + 2 + 2 + 2 * PBX * 2 + 2 + 2 + 2;
-  static constexpr int SMEM_BYTES = 2 * Q_BUFS * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES +
+  static constexpr int SMEM_BYTES = 2 * Q_BUFS * Q_BYTES + SK * K_BYTES + SV * V_BYTES + ONES_BYTES + P_SMEM +
                                     1024 /*bars*/ + 1024 /*align*/;
   // BS: block-scaled P. Every 64-key half of a block carries its own power-of-two
   // scale, applied by the tensor core (kind::mxf8f6f4.block_scale): the codes of
@@ -339,7 +346,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sK = sQ + 2 * C::Q_BUFS * C::Q_BYTES;       // K ring
   const uint32_t sV = sK + C::SK * C::K_BYTES;               // V ring
   const uint32_t sOnes = sV + C::SV * C::V_BYTES;          // RS: e4m3 ones, B columns d_v..d_v+15
-  const uint32_t sBar = sOnes + C::ONES_BYTES;
+  const uint32_t sP = sOnes + C::ONES_BYTES;               // SP: P(t, b) at sP + (PB t + b) P_BYTES
+  const uint32_t sBar = sP + C::P_SMEM;
   uint8_t* bar_ptr = base + (sBar - base_u32);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ptr + 8 * C::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar_ptr + 8 * C::NUM_BARS + 4);
@@ -354,7 +362,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bVFull = bKEmpty + 8 * C::SK;           // [SV] TMA -> PV issuer
   const uint32_t bVEmpty = bVFull + 8 * C::SV;           // [SV] PV issuer -> TMA
   const uint32_t bSFull = bVEmpty + 8 * C::SV;           // [2]  QK issuer -> softmax
-  const uint32_t bSFree = bSFull + 16;                   // [1]  softmax -> QK issuer (128 arrivals; SS)
+  const uint32_t bSFree = bSFull + 16;                   // SS: [1], SP: [2]  softmax -> QK issuer (128 arrivals)
   // P full (softmax -> PV issuer, 128 arrivals) and P done (PV issuer ->
   // softmax), per tile and P buffer. One barrier per
   // buffer keeps a softmax that runs a block ahead from completing two phases of
@@ -379,7 +387,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mbar_init(bQEmpty + 8 * (2 * t + qb), 1);
         }
         mbar_init(bSFull + 8 * t, 1);
-        if (t == 0) mbar_init(bSFree, 128);
+        if (t == 0 || C::SP) mbar_init(bSFree + 8 * t, 128);
         for (int b = 0; b < C::PBX; ++b) {
           mbar_init(bPFull + 8 * (t * C::PBX + b), 128);
           mbar_init(bPDone + 8 * (t * C::PBX + b), 1);
@@ -501,13 +509,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // O_t += P V_s with P from TMEM: buffer pbuf (SS) or the first columns of S_t.
       // RS: the second 128-byte column block of B (leading byte offset) is the
       // ones tile, so the row sums land in O_t's extra columns.
+      // SP: P from shared-memory buffer pbuf (K-major like Q: a K step advances
+      // the start address by 32 bytes).
+      const uint32_t p_lo0 = sdesc_lo(sP, 16);
       auto issue_pv = [&](int t, uint32_t pbuf, uint32_t s, bool accumulate) {
         const uint32_t d = tmem + C::TM_O + t * C::O_STRIDE;
         const uint32_t v_stage = sV + s * C::V_BYTES;
         const uint32_t b_lo = C::RS ? sdesc_lo(v_stage, sOnes - v_stage) : v_lo0 + s * (C::V_BYTES >> 4);
         const uint32_t a_t = tmem + (C::SS ? C::TM_P + pbuf * C::P_COLS : t * 128);
         const uint32_t acc = accumulate ? 1u : 0u;
-        if constexpr (C::BS) {
+        if constexpr (C::SP) {
+          const uint32_t a_lo = p_lo0 + pbuf * (C::P_BYTES >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kBN / C::MMA_K; ++kk)
+            mma_ss_lo<FP8>(d, a_lo + ((kk * C::MMA_K) >> 4), b_lo + ((kk * C::MMA_K * 128) >> 4), C::IDESC_PV,
+                           kk > 0 ? 1u : acc);
+        } else if constexpr (C::BS) {
           // K step kk covers keys 32 kk .. 32 kk + 31 and reads scale byte kk of each row
 #pragma unroll
           for (int kk = 0; kk < kBN / C::MMA_K; ++kk)
@@ -522,6 +539,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
       uint32_t kit = 0, vit = 0;  // K and V ring positions
       uint32_t nq = 0;            // QK^T products issued (SS: uses of the one S buffer)
+      uint32_t nqt[2] = {0, 0};   // SP: uses of S_0 and S_1
       auto take = [&](uint32_t bFull, int nslot, uint32_t& itr, uint32_t& s) -> bool {
         s = itr % nslot;
         const bool r = mbar_wait(bFull + 8 * s, (itr / nslot) & 1, abort_flag);
@@ -532,10 +550,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int u = unit_for(k, blockIdx.x, gridDim.x);
         if (u >= n_units) break;
         const Unit x = decode_unit(u, p);
-        if constexpr (C::SS) {
+        if constexpr (C::SS || C::SP) {
           // Split by role. Warp 1: S = Q_t K_j^T once the softmax has copied the
-          // previous S out. Warp 2: O_t += P_t(j) V_j once the softmax has written
-          // P_t(j) (and rescaled O_t).
+          // previous S out (SS: the one S buffer; SP: S_t). Warp 2:
+          // O_t += P_t(j) V_j once the softmax has written P_t(j) (and rescaled O_t).
           if (warp == 1) {
             const uint32_t qb = C::Q_BUFS == 2 ? (k & 1) : 0;
             const uint32_t qpar = C::Q_BUFS == 2 ? ((k >> 1) & 1) : q_par;
@@ -548,7 +566,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int t = 0; t < 2; ++t) {
                 const int n_t = t ? x.n1 : x.n0;
                 if (j >= n_t) continue;
-                if (nq > 0 && !(ok = mbar_wait(bSFree, (nq - 1) & 1, abort_flag))) break;
+                if constexpr (C::SP) {
+                  if (nqt[t] > 0 && !(ok = mbar_wait(bSFree + 8 * t, (nqt[t] - 1) & 1, abort_flag))) break;
+                  ++nqt[t];
+                } else {
+                  if (nq > 0 && !(ok = mbar_wait(bSFree, (nq - 1) & 1, abort_flag))) break;
+                }
                 trace(kEvQkIssue, nq);
                 ++nq;
                 tc_fence_after();
@@ -779,6 +802,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if constexpr (C::SS) {
           tc_fence_before();
           mbar_arrive(bSFree);  // S may take the next product now
+        } else if constexpr (C::SP) {
+          tc_fence_before();
+          mbar_arrive(bSFree + 8 * t);  // S_t may take this tile's next product now
         }
         if (tracer) trace(kEvSoftmaxHaveS, g);
 
@@ -986,7 +1012,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         l_run += l_blk;
 
-        if constexpr (C::SS) {
+        if constexpr (C::SS || C::SP) {
           // P buffer g % PB is free once PV of block g-PB has completed; O may be
           // rescaled once PV of block g-1 (this unit's previous block) has.
           const uint32_t pb = g % C::PB;
@@ -1018,10 +1044,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               tmem_st16(tO + DV, orr);
             }
           }
-          // P row -> its own TMEM columns (BS: and the row's scales, read by the same PV)
-          tmem_st32(tP + pb * C::P_COLS, sr);
-          if constexpr (C::BS) tmem_st1(tO + C::SF_COL + (warp & 3), sf_word);
-          if constexpr (!FP8) tmem_st32(tP + pb * C::P_COLS + 32, sr + 32);
+          if constexpr (C::SP) {
+            // P row r -> shared memory, K-major with the 128-byte swizzle: 16-byte
+            // chunk c (keys 16c .. 16c + 15) of row r at r * 128 + ((c ^ (r & 7)) << 4)
+            const uint32_t prow = sP + (t * C::PB + pb) * C::P_BYTES + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              st_shared_v4(prow + ((c ^ (r & 7)) << 4), sr[4 * c], sr[4 * c + 1], sr[4 * c + 2], sr[4 * c + 3]);
+            fence_proxy_async_smem();
+          } else {
+            // P row -> its own TMEM columns (BS: and the row's scales, read by the same PV)
+            tmem_st32(tP + pb * C::P_COLS, sr);
+            if constexpr (C::BS) tmem_st1(tO + C::SF_COL + (warp & 3), sf_word);
+            if constexpr (!FP8) tmem_st32(tP + pb * C::P_COLS + 32, sr + 32);
+          }
         } else {
           // rescale this tile's O accumulator (PV_t,i-1 has completed: S_t,i was issued after it)
           if (i > 0 && __any_sync(0xffffffffu, need)) {

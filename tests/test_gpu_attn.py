@@ -60,20 +60,22 @@ SMALL = [
 FP8_P = ["lean", "mufu", "block"]
 
 
-# FP8 with per-head scales has three kernels: both query tiles of a unit on one
-# SM (default), the two tiles on the two SMs of a CTA pair
-# (B200ATTN_FP8_PAIR=1), and one tile per unit on one SM (B200ATTN_FP8_TILE=1);
-# the tests marked with this fixture run all three.
-FP8_KERNELS = ["pair", "two", "tile"]
-FP8_KERNEL_ENV = {"pair": ("0", "1"), "two": ("0", "0"), "tile": ("1", "1")}  # (FP8_TILE, FP8_PAIR)
+# FP8 with per-head scales has four kernel layouts: both query tiles of a unit
+# on one SM sharing one S buffer (default), the same with one S buffer per tile
+# and P in shared memory (B200ATTN_SHARED_S=0), the two tiles on the two SMs of
+# a CTA pair (B200ATTN_FP8_PAIR=1), and one tile per unit on one SM
+# (B200ATTN_FP8_TILE=1); the tests marked with this fixture run all four.
+FP8_KERNELS = ["pair", "two", "tile", "sp"]
+FP8_KERNEL_ENV = {"pair": ("0", "1", "1"), "two": ("0", "0", "1"), "tile": ("1", "1", "1"),
+                  "sp": ("0", "0", "0")}  # (FP8_TILE, FP8_PAIR, SHARED_S)
+FP8_KERNEL_VARS = ("B200ATTN_FP8_TILE", "B200ATTN_FP8_PAIR", "B200ATTN_SHARED_S")
 
 
 @pytest.fixture
 def fp8_kernel(request):
-    old = {k: os.environ.get(k) for k in ("B200ATTN_FP8_TILE", "B200ATTN_FP8_PAIR")}
-    tile, pair = FP8_KERNEL_ENV[request.param]
-    os.environ["B200ATTN_FP8_TILE"] = tile
-    os.environ["B200ATTN_FP8_PAIR"] = pair
+    old = {k: os.environ.get(k) for k in FP8_KERNEL_VARS}
+    for k, v in zip(FP8_KERNEL_VARS, FP8_KERNEL_ENV[request.param]):
+        os.environ[k] = v
     yield request.param
     for k, v in old.items():
         if v is None:
@@ -128,10 +130,14 @@ def lse_atol(fp8_p):
     return MUFU_LSE_ATOL if fp8_p == "mufu" else LEAN_LSE_ATOL
 
 
+@pytest.mark.parametrize("shared_s", ["1", "0"])
 @pytest.mark.parametrize("bf16_p", BF16_P, indirect=True)
 @pytest.mark.parametrize("shape", SMALL)
 @pytest.mark.parametrize("causal", [True, False])
-def test_bf16_matches_oracle(shape, causal, bf16_p):
+def test_bf16_matches_oracle(shape, causal, bf16_p, shared_s, monkeypatch):
+    """BF16 against fp64, with the one shared S buffer (default) and with one S
+    buffer per tile and P over S (B200ATTN_SHARED_S=0)."""
+    monkeypatch.setenv("B200ATTN_SHARED_S", shared_s)
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq))
     o, lse = run_bf16(q, k, v, causal)
@@ -148,7 +154,7 @@ def test_bf16_matches_oracle(shape, causal, bf16_p):
 @pytest.mark.parametrize("causal", [True, False])
 def test_fp8_matches_oracle(shape, causal, fp8_p, fp8_kernel):
     if fp8_p == "block" and fp8_kernel != "two":
-        pytest.skip("block-scaled P is built into the two-tile kernel only")
+        pytest.skip("block-scaled P is built into the two-tile kernel with the shared S buffer only")
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + Hq + 1))
     codes, deq = oracle_fp8_inputs(q, k, v)
@@ -162,12 +168,14 @@ def test_fp8_matches_oracle(shape, causal, fp8_p, fp8_kernel):
 PER_BLOCK_SHAPES = [(1, 4, 2, 300, 128), (2, 2, 1, 700, 128), (1, 4, 4, 520, 192)]
 
 
+@pytest.mark.parametrize("shared_s", ["1", "0"])
 @pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
 @pytest.mark.parametrize("shape", PER_BLOCK_SHAPES)
 @pytest.mark.parametrize("causal", [True, False])
-def test_fp8_per_block_scales_match_oracle(shape, causal, fp8_p):
+def test_fp8_per_block_scales_match_oracle(shape, causal, fp8_p, shared_s, monkeypatch):
     """Scales per (b, h, 128-token block); V blocks get very different magnitudes so the
-    kernel's per-block V reference grows and O is rescaled."""
+    kernel's per-block V reference grows and O is rescaled. Both S-buffer layouts."""
+    monkeypatch.setenv("B200ATTN_SHARED_S", shared_s)
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + 7))
     gain = torch.tensor([0.05, 3.0, 0.5, 20.0, 1.0, 0.01])[(torch.arange(N) // 128) % 6]
@@ -187,12 +195,14 @@ def test_fp8_per_block_scales_match_oracle(shape, causal, fp8_p):
 Q_BLOCK_SHAPES = [(1, 4, 2, 300, 128), (2, 8, 2, 1000, 128), (1, 4, 4, 520, 192)]
 
 
+@pytest.mark.parametrize("shared_s", ["1", "0"])
 @pytest.mark.parametrize("fp8_p", FP8_P, indirect=True)
 @pytest.mark.parametrize("shape", Q_BLOCK_SHAPES)
 @pytest.mark.parametrize("causal", [True, False])
-def test_fp8_q_block_scales_match_oracle(shape, causal, fp8_p):
+def test_fp8_q_block_scales_match_oracle(shape, causal, fp8_p, shared_s, monkeypatch):
     """Q's scales per (b, h, 128-token block), K's and V's per head; Q gets very
-    different magnitudes per block so the per-block scale matters."""
+    different magnitudes per block so the per-block scale matters. Both S-buffer layouts."""
+    monkeypatch.setenv("B200ATTN_SHARED_S", shared_s)
     B, Hq, Hkv, N, dqk = shape
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=N + 11))
     gain = torch.tensor([0.05, 3.0, 0.5, 20.0, 1.0, 0.01])[(torch.arange(N) // 128) % 6]
@@ -365,7 +375,7 @@ def test_bf16_many_units_per_cta(causal, bf16_p):
 @pytest.mark.parametrize("causal", [True, False])
 def test_fp8_many_units_per_cta(causal, fp8_p, fp8_kernel):
     if fp8_p == "block" and fp8_kernel != "two":
-        pytest.skip("block-scaled P is built into the two-tile kernel only")
+        pytest.skip("block-scaled P is built into the two-tile kernel with the shared S buffer only")
     B, Hq, Hkv, N, dqk = MANY_UNITS
     q, k, v = workloads.draw(workloads.gaussian(B, Hq, Hkv, N, dqk, 128, seed=22))
     codes, deq = oracle_fp8_inputs(q, k, v)
@@ -377,10 +387,11 @@ def test_fp8_many_units_per_cta(causal, fp8_p, fp8_kernel):
     assert err <= FP8_TOL, err
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "bf16-mixed", "fp8-lean", "fp8-mufu", "fp8-block", "fp8-lean-pair",
-                                   "fp8-lean-tile"])
+@pytest.mark.parametrize("dtype", ["bf16", "bf16-mixed", "bf16-mixed-sp", "fp8-lean", "fp8-mufu", "fp8-block",
+                                   "fp8-lean-pair", "fp8-lean-tile", "fp8-lean-sp"])
 def test_bitwise_deterministic_over_1000_launches(dtype, monkeypatch):
-    monkeypatch.setenv("B200ATTN_BF16_P", "mixed" if dtype == "bf16-mixed" else "mufu")
+    monkeypatch.setenv("B200ATTN_BF16_P", "mixed" if dtype.startswith("bf16-mixed") else "mufu")
+    monkeypatch.setenv("B200ATTN_SHARED_S", "0" if dtype.endswith("-sp") else "1")
     if dtype.startswith("fp8"):
         monkeypatch.setenv("B200ATTN_FP8_P", dtype.split("-")[1])
         monkeypatch.setenv("B200ATTN_FP8_TILE", "1" if dtype.endswith("-tile") else "0")
@@ -460,7 +471,7 @@ def test_full_size_fp8_sampled(name, hadamard, monkeypatch):
         assert_within(e, FP8_TOL)
 
 
-@pytest.mark.parametrize("fp8_kernel", ["pair", "tile"], indirect=True)
+@pytest.mark.parametrize("fp8_kernel", ["pair", "tile", "sp"], indirect=True)
 @pytest.mark.parametrize("fp8_p", ["lean", "mufu"], indirect=True)
 def test_full_size_fp8_other_kernels_sampled(fp8_p, fp8_kernel):
     """The FP8 kernels other than the default on the full 7B-style layer
