@@ -623,38 +623,93 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
 def measure_e2e(b2, args, w, q_cpu, k_cpu, v_cpu, world, dist_on):
     """Same metric through the public API from pinned host buffers: H2D of Q,K,V, the
-    step (quantizer + attention), D2H of O, all inside the timed region."""
+    step (quantizer + attention), D2H of O, every step inside the timed region.
+
+    Pipelined (the reported value): the H2D of step i+1 and the D2H of step i-1 run on
+    their own CUDA streams while step i computes, on two sets of device buffers; events
+    order each step's copy in -> compute -> copy out and keep a buffer set from being
+    refilled before its previous step has finished with it. The time is from the first
+    H2D to the last D2H, divided by the steps. Serial (reported beside it): copy in,
+    compute and copy out one after another on one stream."""
     hq, hk, hv = q_cpu.pin_memory(), k_cpu.pin_memory(), v_cpu.pin_memory()
     ho = torch.empty((w.B, w.N, w.Hq, w.d_v), dtype=torch.bfloat16).pin_memory()
-    q = torch.empty_like(q_cpu, device="cuda")
-    k = torch.empty_like(k_cpu, device="cuda")
-    v = torch.empty_like(v_cpu, device="cuda")
-    path = Path(b2, q, k, v, args.dtype, args.hadamard, args.fp8_q)
+    sets = []
+    for _ in range(2):
+        q = torch.empty_like(q_cpu, device="cuda")
+        k = torch.empty_like(k_cpu, device="cuda")
+        v = torch.empty_like(v_cpu, device="cuda")
+        sets.append((q, k, v, Path(b2, q, k, v, args.dtype, args.hadamard, args.fp8_q)))
+    steps = max(3, min(args.steps, 10))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
 
-    def step():
+    # serial: one stream
+    def serial_step():
+        q, k, v, path = sets[0]
         q.copy_(hq, non_blocking=True)
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
         path.step()
         ho.copy_(path.o, non_blocking=True)
 
-    steps = max(3, min(args.steps, 10))
-    for _ in range(2):
-        step()
-    torch.cuda.synchronize()
-    if dist_on:
-        torch.distributed.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dist_on)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = ho.numel() * ho.element_size()
+    def timed(run):
+        run(2)  # warm-up
+        torch.cuda.synchronize()
+        if dist_on:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run(steps, e0)
+        e1.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1) / steps, dist_on)
+
+    def run_serial(n, start=None):
+        for _ in range(n):
+            serial_step()
+
+    ms_serial = timed(run_serial)
+
+    # pipelined: copy-in, compute and copy-out streams
+    main = torch.cuda.current_stream()
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+
+    def run_pipelined(n, start=None):
+        in_done, comp_done, out_done = [None, None], [None, None], [None, None]
+        for st in (s_in, s_comp, s_out):
+            st.wait_stream(main)
+        for i in range(n):
+            b = i % 2
+            q, k, v, path = sets[b]
+            with torch.cuda.stream(s_in):
+                if comp_done[b] is not None:
+                    s_in.wait_event(comp_done[b])  # step i-2 has read this set's inputs
+                q.copy_(hq, non_blocking=True)
+                k.copy_(hk, non_blocking=True)
+                v.copy_(hv, non_blocking=True)
+                in_done[b] = ev()
+                in_done[b].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(in_done[b])
+                if out_done[b] is not None:
+                    s_comp.wait_event(out_done[b])  # step i-2's O has been copied out
+                path.step()
+                comp_done[b] = ev()
+                comp_done[b].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[b])
+                ho.copy_(path.o, non_blocking=True)
+                out_done[b] = ev()
+                out_done[b].record(s_out)
+        for st in (s_in, s_comp, s_out):
+            main.wait_stream(st)
+
+    ms = timed(run_pipelined)
     return {"value": world * w.flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "schedule": "pipelined: H2D of step i+1 and D2H of step i-1 overlap step i on separate streams",
+            "serial": {"value": world * w.flops / (ms_serial * 1e-3) / 1e12, "ms_per_step": ms_serial}}
 
 
 def main():
