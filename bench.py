@@ -343,7 +343,7 @@ def fp8_p_desc(args) -> str:
     env_p = os.environ.get("B200ATTN_FP8_P")
     if env_p == "mufu":
         return "mufu"
-    if env_p == "lean" or args.fp8_q == "fused" or os.environ.get("B200ATTN_SHARED_S") == "0":
+    if env_p == "lean" or os.environ.get("B200ATTN_SHARED_S") == "0":
         return "lean"
     return "lean, block-scaled (power-of-two scale per 64-key half block)"
 
@@ -505,7 +505,7 @@ def kernel_name(dtype: str, w: workloads.Workload, fused_q: bool = False) -> str
     """The attention kernel (and probability mode) the library runs for this call."""
     env_p = os.environ.get("B200ATTN_FP8_P")
     if dtype == "fp8" and fused_q:
-        fp8_p = "mufu" if env_p == "mufu" else "lean"
+        fp8_p = env_p if env_p in ("lean", "mufu") else "lean,block-scaled"
         return f"attn_fwd_kernel<{w.d_qk},{w.d_v},fp8,{fp8_p},fused-q>"
     if dtype == "fp8":
         fp8_p = "mufu" if env_p == "mufu" else "lean"

@@ -212,9 +212,10 @@ struct AttnCfg {
   static_assert(!BSP || (FP8 && FMA_P && RS), "block-scaled P is a variant of Lean P with tensor-core row sums");
   static_assert(!BS || SFB_COLS >= 8, "B scales need the columns n / 32 of N = d_v + 16");
   // Register split. The block-scaled PV issue with d_qk = 192 needs a few more
-  // registers in the issuer warps than 72 (it spilled there); its softmax fits in 200.
-  static constexpr int REGS_LOW = BS && DQK > 128 ? 80 : kRegsLow;
-  static constexpr int REGS_HIGH = BS && DQK > 128 ? 200 : kRegsHigh;
+  // registers in the issuer warps than 72 (it spilled there); its softmax fits in
+  // 200, unless it also encodes Q (QF), which keeps 208.
+  static constexpr int REGS_LOW = BS && DQK > 128 && !QF ? 80 : kRegsLow;
+  static constexpr int REGS_HIGH = BS && DQK > 128 && !QF ? 200 : kRegsHigh;
   static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= kAttnThreads * kRegsAtLaunch, "register split");
   static_assert(DV == 128, "TMEM budget assumes d_v = 128");
   static_assert(SK >= 2 && SV >= 1, "K/V rings");

@@ -83,7 +83,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // call so A/B runs need no rebuild):
 //  * block (default): Lean P with one power-of-two scale per 64-key half block,
 //    applied by the block-scaled MMA. Built into the two-tile kernel with
-//    per-head K/V scales; the other configurations run Lean P. Paired A/B
+//    per-head K/V scales (Q per head, per block or quantised in the kernel); the
+//    other configurations run Lean P. Paired A/B
 //    against Lean P on B200: 1-2% faster at 16K-32K with d = 128, within 1% on
 //    the other shapes, and more accurate (no probability of a row drops out of
 //    e4m3's range because another half block holds the row's maximum).
@@ -432,6 +433,11 @@ int b200attn_fwd_fp8_fused_q(const void* q, const void* k, const void* v, void* 
   p.q_codes_out = static_cast<uint8_t*>(q_fp8_out);
   p.q_scale_out = q_scale_out;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fp8_block_scaled_p()) {
+    if (d_qk == 128)
+      return launch_attn_t<128, 128, true, true, true, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+    return launch_attn_t<192, 128, true, true, true, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
+  }
   if (fp8_lean_p()) {
     if (d_qk == 128) return launch_attn_t<128, 128, true, true, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);
     return launch_attn_t<192, 128, true, true, true, true>(q, k, v, p, d_qk, d_v, sm_count, st);

@@ -138,6 +138,8 @@ int b200attn_fwd(const void* q, const void* k, const void* v, void* o,
  * q_scale_out  optional (NULL allowed) device fp32 [B, Hq, ceil(N/128)]:
  *        receives the scales the kernel used
  * Other arguments as in b200attn_fwd (o bf16 [B, N, Hq, d_v], optional lse).
+ * Probabilities are formed as by b200attn_fwd with per-head K/V scales
+ * (block-scaled Lean P unless B200ATTN_FP8_P selects another mode).
  *
  * Errors: INVALID (as b200attn_fwd; missing k/v scales; hadamard not 0/1;
  * misaligned outputs), UNSUPPORTED, CUDA.

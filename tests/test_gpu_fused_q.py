@@ -55,7 +55,7 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("fp8_p", ["lean", "mufu"])
+@pytest.mark.parametrize("fp8_p", ["lean", "mufu", "block"])
 @pytest.mark.parametrize("hadamard", [False, True])
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("causal", [True, False])
