@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import math
 import os
 import statistics
@@ -91,12 +92,23 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(src: str) -> str:
+    """C/C++ source without its comments and blank space, so that the hash below
+    changes with the code and not with its comments (the sources hold no comment
+    markers inside string literals)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_sources_sha() -> str:
+    """Hash of the attention kernels' code (comments and blank space left out): the
+    DRAM traffic figures in profiles/ are valid only for the code they were taken on."""
     h = hashlib.sha256()
     for f in ("attn_fwd_kernel.cuh", "attn_fwd_pair_kernel.cuh", "attn_fwd_tile_kernel.cuh", "sm100_ptx.cuh",
               "q_encode.cuh", "attn_trace.cuh"):
-        with open(os.path.join(ROOT, "bf16_causal_prefill_fwd_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "bf16_causal_prefill_fwd_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

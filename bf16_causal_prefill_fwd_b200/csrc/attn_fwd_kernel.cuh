@@ -17,8 +17,8 @@
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer of Q tiles and of the K ring
-//   warps 1, 2  MMA issuers (one thread each; warp 2 only with SHARED_S),
-//               see below
+//   warps 1, 2  MMA issuers (one thread each; warp 2 only with SHARED_S and
+//               in the FP8 private-S layout), see below
 //   warp 3      TMA producer of the V ring
 //   warps 4-7   softmax + epilogue for tile 0 (one thread per query row)
 //   warps 8-11  softmax + epilogue for tile 1
@@ -46,9 +46,16 @@
 //    warp 2 every PV (each waits for its P), so neither wait holds up the
 //    other's MMAs.
 //  * otherwise: [0,128) S_0, [128,256) S_1, [256,384) O_0, [384,512) O_1, with
-//    P written over the first columns of S_t; S_t for the next block can only
-//    start after PV_t has read P, so warp 1 alone issues PV_t then QK_t for
-//    each tile in turn (one thread's MMAs run in issue order).
+//    bf16: P written over the first columns of S_t; S_t for the next block can
+//    only start after PV_t has read P, so warp 1 alone issues PV_t then QK_t
+//    for each tile in turn (one thread's MMAs run in issue order).
+//    e4m3 ("private S", SP): P goes to shared memory (two buffers per tile) and
+//    PV reads it there, so a tile's next QK^T waits only for its own S
+//    copy-out; two issuers as in SHARED_S; row sums in registers.
+//  * e4m3 with per-head K/V scales and SHARED_S: P may be block-scaled (BSP):
+//    each 64-key half of a block carries its own power-of-two scale, held as
+//    UE8M0 bytes in the spare columns of O_t and applied by
+//    tcgen05.mma.kind::mxf8f6f4.block_scale (see AttnCfg).
 //
 // Online softmax per row (log2 domain, c = s * log2(e) [* q/k scales]):
 //   m_blk = max_j S_ij; m_new = max(m_run, c * m_blk)
@@ -57,7 +64,9 @@
 //   O = O_acc / l at the end.
 // T lets the running max lag the true one (P <= 2^(T+E)), which skips most O
 // rescales; E shifts FP8 probabilities up so the e4m3 normal range covers more
-// binades. Both cancel exactly in O_acc / l.
+// binades. Both cancel exactly in O_acc / l. With block-scaled P the codes of
+// each half block are shifted by their own integer instead, so T is bounded
+// only by the fp32 growth of O and l.
 //
 // Probabilities on the FMA pipe (template switch FMA_P, chosen on the host):
 // for FP8 it selects Lean P below; for BF16 it sends one score in four through
