@@ -97,3 +97,34 @@ def test_reference_arm_line_on_rank_zero(capsys):
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["steps"] == 1 and line["warmup"] == 3 and line["dtype"] == "f64"
+
+
+def test_kernel_hash_ignores_comments_and_follows_code():
+    """The traffic figures are keyed to a hash of the kernel code: a comment or
+    blank-space edit leaves it unchanged, a code edit changes it."""
+    import bench
+    code = "int f(int x) {\n  return x + 1;  // add one\n}\n/* block\n comment */\n"
+    assert bench._code_only(code) == bench._code_only("int f(int x) { return x + 1; }")
+    assert bench._code_only(code) != bench._code_only("int f(int x) { return x + 2; }")
+    assert len(bench.kernel_sources_sha()) == 16
+
+
+@pytest.mark.parametrize("env,fused,expect", [
+    ({}, False, "attn_fwd_kernel<128,128,fp8,lean,block-scaled>"),
+    ({"B200ATTN_FP8_P": "lean"}, False, "attn_fwd_kernel<128,128,fp8,lean>"),
+    ({"B200ATTN_FP8_P": "mufu"}, False, "attn_fwd_kernel<128,128,fp8,mufu>"),
+    ({"B200ATTN_SHARED_S": "0"}, False, "attn_fwd_kernel<128,128,fp8,lean,private-S>"),
+    ({"B200ATTN_FP8_PAIR": "1"}, False, "attn_fwd_pair_kernel<128,128,fp8,lean>"),
+    ({"B200ATTN_FP8_TILE": "1"}, False, "attn_fwd_tile_kernel<128,128,fp8,lean>"),
+    ({}, True, "attn_fwd_kernel<128,128,fp8,lean,block-scaled,fused-q>"),
+    ({"B200ATTN_FP8_P": "mufu"}, True, "attn_fwd_kernel<128,128,fp8,mufu,fused-q>"),
+])
+def test_kernel_name_follows_the_library_dispatch(env, fused, expect, monkeypatch):
+    """bench.py names the kernel the library runs for the FP8 step under each switch."""
+    import bench
+    import workloads
+    for k in ("B200ATTN_FP8_P", "B200ATTN_SHARED_S", "B200ATTN_FP8_PAIR", "B200ATTN_FP8_TILE"):
+        monkeypatch.delenv(k, raising=False)
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    assert bench.kernel_name("fp8", workloads.gqa7b(), fused_q=fused) == expect
