@@ -70,6 +70,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-dtype", action="store_true", help="skip the secondary dtype measurement")
     ap.add_argument("--no-at-32k", action="store_true", help="skip the N=32768 (B=1) Gaussian layer")
+    ap.add_argument("--varlen", action="store_true",
+                    help="measure the packed variable-length path instead (b200attn_fwd_varlen): 24 causal "
+                         "sequences with log-uniform lengths in [256, 8192], 7B-style heads; one JSON line")
     ap.add_argument("--measure-peaks", action="store_true",
                     help="print the bf16 and e4m3 GEMM tensor peaks of this GPU as JSON and exit")
     return ap.parse_args()
@@ -724,6 +727,89 @@ def measure_e2e(b2, args, w, q_cpu, k_cpu, v_cpu, world, dist_on):
             "serial": {"value": world * w.flops / (ms_serial * 1e-3) / 1e12, "ms_per_step": ms_serial}}
 
 
+def varlen_lengths(n_seq: int = 24, lo: int = 256, hi: int = 8192, seed: int = 5) -> list:
+    """Sequence lengths of the packed-batch workload: log-uniform in [lo, hi], seeded."""
+    g = torch.Generator().manual_seed(seed)
+    u = torch.rand(n_seq, generator=g, dtype=torch.float64)
+    return [int(x) for x in (lo * (hi / lo) ** u).round().tolist()]
+
+
+class VarlenPath:
+    """One step of the packed variable-length path: the quantizer over the packed
+    tensors (per-head scales), then b200attn_fwd_varlen; or BF16 attention alone."""
+
+    def __init__(self, b2, q, k, v, cu, dtype: str):
+        self.b2, self.q, self.k, self.v, self.cu, self.dtype = b2, q, k, v, cu, dtype
+        total, Hq, dqk = q.shape
+        Hkv, dv = k.shape[1], v.shape[2]
+        dev = q.device
+        self.o = torch.empty((total, Hq, dv), dtype=torch.bfloat16, device=dev)
+        self.vws = torch.empty(max(int(b2.load_library().b200attn_fwd_varlen_workspace_bytes(cu.numel() - 1, total, Hq)), 16),
+                               dtype=torch.uint8, device=dev)
+        if dtype == "fp8":
+            self.q8 = torch.empty((1,) + tuple(q.shape), dtype=torch.float8_e4m3fn, device=dev)
+            self.k8 = torch.empty((1,) + tuple(k.shape), dtype=torch.float8_e4m3fn, device=dev)
+            self.v8 = torch.empty((1,) + tuple(v.shape), dtype=torch.float8_e4m3fn, device=dev)
+            self.sq = torch.empty((1, Hq), dtype=torch.float32, device=dev)
+            self.sk = torch.empty((1, Hkv), dtype=torch.float32, device=dev)
+            self.sv = torch.empty((1, Hkv), dtype=torch.float32, device=dev)
+            self.qws = torch.empty(max(b2.quantize_qkv_workspace_bytes(1, total, Hq, Hkv, "head"), 4),
+                                   dtype=torch.uint8, device=dev)
+        self.launches_per_step = 4 if dtype == "fp8" else 2  # quantizer passes, unit-table builder, attention
+
+    def step(self, ev_a0=None, ev_a1=None):
+        b2 = self.b2
+        if self.dtype == "fp8":
+            b2.quantize_qkv_fp8(self.q.unsqueeze(0), self.k.unsqueeze(0), self.v.unsqueeze(0), granularity="head",
+                                workspace=self.qws, out=(self.q8, self.sq, self.k8, self.sk, self.v8, self.sv))
+            if ev_a0 is not None:
+                ev_a0.record()
+            b2.attn_varlen_fwd(self.q8[0], self.k8[0], self.v8[0], self.cu, q_scale=self.sq[0], k_scale=self.sk[0],
+                               v_scale=self.sv[0], out=self.o, workspace=self.vws)
+        else:
+            if ev_a0 is not None:
+                ev_a0.record()
+            b2.attn_varlen_fwd(self.q, self.k, self.v, self.cu, out=self.o, workspace=self.vws)
+        if ev_a1 is not None:
+            ev_a1.record()
+
+
+def run_varlen(args, local_rank: int):
+    """The packed variable-length path on one GPU: FP8 step and BF16 attention, each
+    timed like the main step (CUDA events, L2 flushed between steps)."""
+    import bf16_causal_prefill_fwd_b200 as b2
+    torch.cuda.set_device(local_rank)
+    lens = varlen_lengths()
+    Hq, Hkv, d = 32, 8, 128
+    total = sum(lens)
+    g = torch.Generator().manual_seed(6)
+    q = torch.randn(total, Hq, d, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(total, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(total, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device="cuda")
+    flops = float(sum(n * n for n in lens)) * Hq * (d + d)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    out = {}
+    for dtype in ("fp8", "bf16"):
+        path = VarlenPath(b2, q, k, v, cu, dtype)
+        with ClockSampler(local_rank) as clk:
+            step_ms, attn_ms = time_path(path, args.steps, args.warmup, args.settle_s, flush, False, clk)
+        assert b2.check() == 0
+        ms, ams = statistics.mean(step_ms), statistics.mean(attn_ms)
+        out[dtype] = {"value": flops / (ms * 1e-3) / 1e12, "ms_per_step": ms,
+                      "kernel_tflops": flops / (ams * 1e-3) / 1e12, "kernel_ms": ams, "clocks": clk.summary()}
+    line = {"metric": "packed variable-length causal prefill attn TFLOP/s", "value": out["fp8"]["value"],
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": out["fp8"]["ms_per_step"], "higher_is_better": True, "dtype": "fp8_e4m3",
+            "data": "synthetic", "fp8": out["fp8"], "bf16": out["bf16"],
+            "config": {"workload": f"varlen: {len(lens)} causal sequences, lengths log-uniform in [256, 8192] "
+                                   f"(seed 5), {total} tokens, Hq={Hq} Hkv={Hkv} d={d}",
+                       "lengths": lens, "flops_per_step": flops, "flop_convention": "sum_b n_b^2 * Hq * (d_qk + d_v)",
+                       "step": "e4m3 quantizer (per-head scales) on the packed tensors + b200attn_fwd_varlen",
+                       "l2": "256 MiB buffer written between timed steps (untimed)"}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     if args.warmup < 3:
@@ -739,6 +825,9 @@ def main():
     if args.measure_peaks:
         torch.cuda.set_device(local_rank)
         print(json.dumps(measure_tensor_peaks()), flush=True)
+        return
+    if args.varlen:
+        run_varlen(args, local_rank)
         return
     dist_on = world > 1
     if dist_on:
