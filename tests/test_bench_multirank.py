@@ -128,3 +128,12 @@ def test_kernel_name_follows_the_library_dispatch(env, fused, expect, monkeypatc
     for k, v in env.items():
         monkeypatch.setenv(k, v)
     assert bench.kernel_name("fp8", workloads.gqa7b(), fused_q=fused) == expect
+
+
+def test_varlen_workload_recipe_is_fixed():
+    """bench.py --varlen: 24 seeded log-uniform lengths in [256, 8192]; the same on every call."""
+    import bench
+    a, b = bench.varlen_lengths(), bench.varlen_lengths()
+    assert a == b and len(a) == 24
+    assert all(256 <= n <= 8192 for n in a)
+    assert a != bench.varlen_lengths(seed=6)
