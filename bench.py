@@ -591,7 +591,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         other["dtype"] = other_dtype
         other["clocks"] = clk_o.summary()
 
-    # The spec point: the Gaussian sweep's N = 32768 (B = 1) layer, both dtypes.
+    # The target point: the Gaussian sweep's N = 32768 (B = 1) layer, both dtypes.
     at_32k = None
     if not args.no_at_32k and w.name != "sweep32768":
         w32 = workloads.sweep(32768)
