@@ -231,6 +231,60 @@ __device__ __forceinline__ void encode_body(const __nv_bfloat16* __restrict__ x,
     return;
   }
   using L = QuantLayout<D>;
+  if constexpr (D == 128 && HAD) {
+    // Rotated d = 128 rows: the rotated values (64 registers) stay in registers
+    // between the absmax and the encode, so each row is rotated once.
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, sub = lane >> 4;
+    uint4 raw[L::ITERS];
+#pragma unroll
+    for (int it = 0; it < L::ITERS; ++it) {
+      const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
+      const int rc = row < N ? row : N - 1;
+      raw[it] = load_lane_raw<D>(x + (static_cast<size_t>(b) * N + rc) * H * D + static_cast<size_t>(h) * D, lane);
+    }
+#pragma unroll
+    for (int it = 0; it < L::ITERS; ++it)
+      asm volatile("" : "+r"(raw[it].x), "+r"(raw[it].y), "+r"(raw[it].z), "+r"(raw[it].w));
+    float v[L::ITERS][8];
+    float m = 0.0f;
+#pragma unroll
+    for (int it = 0; it < L::ITERS; ++it) {
+      lane_values<D, HAD>(raw[it], lane, v[it]);
+      if (blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub < N) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[it][e]));
+      }
+    }
+    if constexpr (PER_HEAD) {
+      m = 0.0f;
+      const float* ph = partial + (static_cast<size_t>(b) * H + h) * nblk;
+      for (int i = threadIdx.x; i < nblk; i += kQuantThreads) m = fmaxf(m, ph[i]);
+    }
+    const float amax = block_max(m, red);
+    const bool pos = amax > 0.0f;
+    const float inv = pos ? __fdiv_rn(448.0f, amax) : 1.0f;
+    const float sc = pos ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    if (threadIdx.x == 0) {
+      if (PER_HEAD) {
+        if (blk == 0) scale[static_cast<size_t>(b) * H + h] = sc;
+      } else {
+        scale[(static_cast<size_t>(b) * H + h) * nblk + blk] = sc;
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < L::ITERS; ++it) {
+      const int row = blk * kQuantBlock + warp * 16 + it * L::ROWS_PER_INSTR + sub;
+      if (row < N) {
+        uint32_t c[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          c[q] = pack_e4m3x2(__fmul_rn(v[it][2 * q], inv), __fmul_rn(v[it][2 * q + 1], inv));
+        *reinterpret_cast<uint2*>(y + (static_cast<size_t>(b) * N + row) * H * D + static_cast<size_t>(h) * D +
+                                  8 * (lane & 15)) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+      }
+    }
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint4 raw[L::ITERS];
   float m;
