@@ -674,26 +674,26 @@ def measure_e2e(b2, args, w, q_cpu, k_cpu, v_cpu, world, dist_on):
             torch.distributed.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        run(steps, e0)
+        run(steps)
         e1.record()
         torch.cuda.synchronize()
         return max_over_ranks(e0.elapsed_time(e1) / steps, dist_on)
 
-    def run_serial(n, start=None):
+    def run_serial(n):
         for _ in range(n):
             serial_step()
 
     ms_serial = timed(run_serial)
 
     # pipelined: copy-in, compute and copy-out streams
-    main = torch.cuda.current_stream()
+    origin = torch.cuda.current_stream()
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
 
-    def run_pipelined(n, start=None):
+    def run_pipelined(n):
         in_done, comp_done, out_done = [None, None], [None, None], [None, None]
         for st in (s_in, s_comp, s_out):
-            st.wait_stream(main)
+            st.wait_stream(origin)
         for i in range(n):
             b = i % 2
             q, k, v, path = sets[b]
@@ -718,7 +718,7 @@ def measure_e2e(b2, args, w, q_cpu, k_cpu, v_cpu, world, dist_on):
                 out_done[b] = ev()
                 out_done[b].record(s_out)
         for st in (s_in, s_comp, s_out):
-            main.wait_stream(st)
+            origin.wait_stream(st)
 
     ms = timed(run_pipelined)
     return {"value": world * w.flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
